@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA weight-absorbed decode step on B200.
+
+A step is the whole hot path over one batch: append the step's n_q new tokens
+to the latent cache (mla_append_cache), absorb W^UK into the queries
+(mla_absorb_q), attend against the cache (mla_decode_attend) and merge the
+split partials + apply W^UV (mla_decode_finish).  Inputs are seeded synthetic
+tensors of the configuration's shapes (mla_inputs); the cache is filled before
+timing and stays resident in HBM.  L2 is flushed (a 256 MiB write) between
+timed steps.
+
+  python bench.py [--config v2] [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  With --gpus N > 1 (torchrun), every rank runs
+its own batch (weak scaling, no data-path collective); timing is the max over
+ranks.  --impl reference times the fp64 CPU oracle on a bounded sample.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mla_inputs as mi  # noqa: E402
+
+METRIC = "MLA absorbed decode: µs/step, TB/s & TFLOP/s as % of B200 roofline"
+UNIT = "TB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# kernels each C-ABI call of the step launches
+KERNELS_PER_STEP = {"append": 1, "absorb": 1, "attend": 1, "finish": 1}
+CORE_SOURCES = ["mla_latent_kv_34_b200/csrc/decode_simt.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="v2", choices=sorted(mi.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ workload arithmetic
+
+def step_counts(cfg: mi.MLAConfig, lengths: np.ndarray) -> dict:
+    """Algorithmic bytes / FLOPs of one step (minimum traffic of the documented calls)."""
+    H, T, n_q = cfg.H, cfg.T, cfg.n_q
+    sum_L = int(lengths.sum())
+    cache = sum_L * mi.D_ROW * 2
+    weights = 2 * H * mi.D_H * mi.D_C * 2
+    q_in = T * H * (mi.D_H + mi.D_R) * 2
+    q_abs = 2 * T * H * mi.D_ROW * 2            # written by absorb, read by attend
+    out = T * H * mi.D_H * 2
+    new_rows = T * mi.D_ROW * 2 * 2              # raw rows read + packed rows written
+    core_flops = 2 * n_q * H * (mi.D_ROW + mi.D_C) * sum_L
+    proj_flops = 2 * 2 * T * H * mi.D_H * mi.D_C  # absorb + up-projection
+    return {
+        "sum_L": sum_L,
+        "core_bytes": cache,                      # per cached token: 1152 B
+        "core_flops": core_flops,                 # per cached token: 2 n_q H (576 + 512)
+        "step_bytes": cache + weights + q_in + q_abs + out + new_rows,
+        "step_flops": core_flops + proj_flops,
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(config_name: str, launch_units: int):
+    """DRAM bytes per launch of the core kernel from a committed ncu summary, if current."""
+    p = os.path.join(ROOT, "profiles", "decode_core_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_hash") != source_hash(CORE_SOURCES):
+        return None
+    ent = d.get("per_config", {}).get(config_name)
+    if not ent:
+        return None
+    # scaled by cached tokens processed when captured on a smaller case
+    return float(ent["dram_bytes_per_launch"]) * launch_units / float(ent["units"])
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append({"sm": float(parts[2]), "max": float(parts[3]), "power": float(parts[4]),
+                             "hw": parts[6], "hwt": parts[7], "swt": parts[8], "pcap": parts[9]})
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                            ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["max"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows), "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+class Dist:
+    def __init__(self, gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+        if gpus > 1 and self.world != gpus:
+            raise SystemExit(f"--gpus {gpus} needs torchrun with {gpus} processes (WORLD_SIZE={self.world})")
+
+    def init(self, torch):
+        torch.cuda.set_device(self.local_rank)
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local_rank))
+            self.pg = True
+
+    def barrier(self, torch):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[self.local_rank])
+
+    def reduce(self, torch, value: float, op: str) -> float:
+        if not self.pg:
+            return value
+        import torch.distributed as dist
+        t = torch.tensor([value], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ our arm
+
+def build_state(torch, mla, cfg: mi.MLAConfig, dev):
+    lengths = mi.kv_lengths(cfg)
+    starts = mi.seq_starts(lengths)
+    N = int(lengths.sum())
+
+    def dbf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    cache = torch.zeros((N, mi.D_ROW), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    rope = mla.rope_table(int(lengths.max()), cfg.rope_base, dev)
+    seq_start = torch.from_numpy(starts).to(dev)
+    seq_of_row = np.repeat(np.arange(cfg.B, dtype=np.int32), lengths)
+    pos_of_row = (np.arange(N, dtype=np.int64) - np.repeat(starts, lengths)).astype(np.int32)
+    chunk = 1 << 18
+    for r0 in range(0, N, chunk):
+        n = min(chunk, N - r0)
+        c, k = mi.token_rows(cfg, r0, n)
+        mla.append_cache(cache, seq_start, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
+                         torch.from_numpy(pos_of_row[r0:r0 + n]).to(dev), dbf(c), dbf(k), rope, status)
+    # the step's new tokens: the last n_q rows of every sequence
+    new_rows = np.concatenate([starts[b] + lengths[b] - cfg.n_q + np.arange(cfg.n_q) for b in range(cfg.B)])
+    new_c = np.concatenate([mi.token_rows(cfg, int(r), 1)[0] for r in new_rows])
+    new_k = np.concatenate([mi.token_rows(cfg, int(r), 1)[1] for r in new_rows])
+    new_seq = np.repeat(np.arange(cfg.B, dtype=np.int32), cfg.n_q)
+    new_pos = pos_of_row[new_rows].astype(np.int32)
+    qn, qr = mi.queries(cfg)
+    host = {  # pinned host copies of the per-step inputs (for the end-to-end leg)
+        "c_kv": torch.from_numpy(new_c.view(np.int16)).view(torch.bfloat16).pin_memory(),
+        "k_rope": torch.from_numpy(new_k.view(np.int16)).view(torch.bfloat16).pin_memory(),
+        "seq_idx": torch.from_numpy(new_seq).pin_memory(),
+        "pos": torch.from_numpy(new_pos).pin_memory(),
+        "q_nope": torch.from_numpy(qn.view(np.int16)).view(torch.bfloat16).pin_memory(),
+        "q_rope": torch.from_numpy(qr.view(np.int16)).view(torch.bfloat16).pin_memory(),
+    }
+    devt = {k: v.to(dev) for k, v in host.items()}
+    T, H = cfg.T, cfg.H
+    st = {
+        "lengths": lengths, "cache": cache, "status": status, "rope": rope, "seq_start": seq_start,
+        "kv_len": torch.from_numpy(lengths.astype(np.int32)).to(dev),
+        "W_UK": dbf(mi.weights(cfg, "uk")), "W_UV": dbf(mi.weights(cfg, "uv")),
+        "host": host, "dev": devt,
+        "q_abs": torch.empty((T, H, mi.D_ROW), dtype=torch.bfloat16, device=dev),
+        "out": torch.empty((T, H, mi.D_H), dtype=torch.bfloat16, device=dev),
+        "out_host": torch.empty((T, H, mi.D_H), dtype=torch.bfloat16).pin_memory(),
+        "ws": torch.empty(mla.decode_workspace_bytes(cfg.B, cfg.n_q, H, 0), dtype=torch.uint8, device=dev),
+    }
+    torch.cuda.synchronize()
+    return st
+
+
+def run_step(mla, cfg, st, ev=None):
+    d = st["dev"]
+    if ev:
+        ev[0].record()
+    mla.append_cache(st["cache"], st["seq_start"], d["seq_idx"], d["pos"], d["c_kv"], d["k_rope"], st["rope"],
+                     st["status"])
+    mla.absorb_q(d["q_nope"], d["q_rope"], d["pos"], st["W_UK"], st["rope"], q_out=st["q_abs"],
+                 dev_status=st["status"])
+    if ev:
+        ev[1].record()
+    mla.decode_attend(st["q_abs"], st["cache"], st["seq_start"], st["kv_len"], cfg.n_q, cfg.scale, 0, st["ws"],
+                      dev_status=st["status"])
+    if ev:
+        ev[2].record()
+    mla.decode_finish(st["W_UV"], cfg.B, cfg.n_q, 0, st["ws"], st["out"])
+    if ev:
+        ev[3].record()
+
+
+def run_ours(args, dist):
+    import torch
+    dist.init(torch)
+    import mla_latent_kv_34_b200 as mla
+    dev = torch.device("cuda", dist.local_rank)
+    base = mi.CONFIGS[args.config]
+    cfg = mi.MLAConfig(**{**base.__dict__, "seed": base.seed + 7919 * dist.rank})
+    st = build_state(torch, mla, cfg, dev)
+    counts = step_counts(cfg, st["lengths"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        run_step(mla, cfg, st)
+    torch.cuda.synchronize()
+    if int(st["status"].item()) != 0:
+        raise SystemExit(f"device status {mla.device_status_string(int(st['status'].item()))}")
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = None if args.no_clocks else ClockSampler(uuid)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    dist.barrier(torch)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        run_step(mla, cfg, st, evs[i])
+    torch.cuda.synchronize()
+    dist.barrier(torch)
+    clocks = sampler.stop() if sampler else None
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    core_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = dist.reduce(torch, sum(step_ms), "max")
+    core_mean_ms = dist.reduce(torch, statistics.mean(core_ms), "max")
+    ms_per_step = total_ms / args.steps
+    bytes_all = dist.reduce(torch, float(counts["step_bytes"]), "sum")
+    flops_all = dist.reduce(torch, float(counts["step_flops"]), "sum")
+    value = bytes_all / (ms_per_step * 1e-3) / 1e12
+
+    # end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h, d = st["host"], st["dev"]
+        h2d = sum(t.numel() * t.element_size() for t in h.values())
+        d2h = st["out_host"].numel() * st["out_host"].element_size()
+        ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        dist.barrier(torch)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            ee[i][0].record()
+            for k in h:
+                d[k].copy_(h[k], non_blocking=True)
+            run_step(mla, cfg, st)
+            st["out_host"].copy_(st["out"], non_blocking=True)
+            ee[i][1].record()
+        torch.cuda.synchronize()
+        dist.barrier(torch)
+        e2e_ms = dist.reduce(torch, sum(e[0].elapsed_time(e[1]) for e in ee), "max") / args.steps
+        e2e = {"value": round(bytes_all / (e2e_ms * 1e-3) / 1e12, 4), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    if int(st["status"].item()) != 0:
+        raise SystemExit(f"device status {mla.device_status_string(int(st['status'].item()))}")
+
+    peaks, peak_src = load_peaks()
+    core_s = core_mean_ms * 1e-3
+    t_bytes = counts["core_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_flops = counts["core_flops"] / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_bytes >= t_flops else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = counts["core_bytes"] / core_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = counts["core_flops"] / core_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    roofline = {
+        "kernel": "mla_decode_attend", "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+        "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} (burst)",
+        "traffic": traffic_for(args.config, counts["sum_L"]),
+        "algorithmic_bytes": counts["core_bytes"], "algorithmic_flops": counts["core_flops"],
+        "us_per_launch": round(core_mean_ms * 1e3, 3),
+        "tflops_achieved": round(counts["core_flops"] / core_s / 1e12, 2),
+        "hbm_gbs_achieved": round(counts["core_bytes"] / core_s / 1e9, 1),
+        "frac_vs_sustained_tensor": round(
+            max(t_bytes, counts["core_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)) / core_s, 4),
+    }
+    step_roof_s = max(counts["step_bytes"] / (peaks["hbm_gbs"] * 1e9), counts["step_flops"] / (peaks["bf16_tflops"] * 1e12))
+
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, mla_inputs)",
+        "config": {"workload": f"{cfg.name}: B={cfg.B} H={cfg.H} n_q={cfg.n_q} "
+                               f"L={'U[1,%d]' % cfg.L_max if cfg.L is None else cfg.L} d_c=512 d_R=64 d_h=128",
+                   "B": cfg.B, "H": cfg.H, "n_q": cfg.n_q, "sum_L": counts["sum_L"],
+                   "step": "append + absorb_q + decode_attend + decode_finish",
+                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"dp{args.gpus} (replicas)"},
+        "us_per_step": round(ms_per_step * 1e3, 2),
+        "tflops": round(flops_all / (ms_per_step * 1e-3) / 1e12, 2),
+        "cache_tokens_per_s": round(dist.reduce(torch, float(counts["sum_L"]), "sum") / (ms_per_step * 1e-3), 1),
+        "step_roofline_frac": round(step_roof_s / (ms_per_step * 1e-3), 4),
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": sum(KERNELS_PER_STEP.values()) * args.steps,
+        "clocks": clocks,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, st["lengths"], counts, args.cpu_seconds)
+    dist.close()
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ the oracle as baseline / reference arm
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(cfg, lengths, heads, b=0):
+    """Run the fp64 naive oracle on sequence b, the given heads; returns seconds."""
+    from oracle import naive as on
+    s = mi.sequence(cfg, b, lengths)
+    f = mi.bf16_bits_to_f64
+    Wk, Wv = f(mi.weights(cfg, "uk")), f(mi.weights(cfg, "uv"))
+    args = (f(s.c_kv), f(s.k_rope), f(s.q_nope), f(s.q_rope), Wk, Wv, cfg.n_q)
+    t = time.perf_counter()
+    on.attend_naive(*args, scale=cfg.scale, base=cfg.rope_base, heads=heads)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(cfg, lengths, counts, target_s: float):
+    b = int(np.argmax(lengths))
+    t1 = oracle_sample(cfg, lengths, [0], b)
+    nh = int(max(1, min(cfg.H, target_s / max(t1, 1e-6))))
+    heads = list(range(nh))
+    t = oracle_sample(cfg, lengths, heads, b)
+    # extrapolate per (cached token x head): the oracle's cost is linear in both
+    per_unit = t / (int(lengths[b]) * nh)
+    full_s = per_unit * counts["sum_L"] * cfg.H
+    return {"value": round(counts["step_bytes"] / full_s / 1e12, 8), "unit": UNIT, "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"sequence {b} (L={int(lengths[b])}), {nh}/{cfg.H} heads, {t:.1f} s; "
+                      f"extrapolated to the full step per (cached token x head): {full_s:.1f} s/step"}
+
+
+def run_reference(args, dist):
+    if dist.rank != 0:
+        return
+    base = mi.CONFIGS[args.config]
+    cfg = base
+    lengths = mi.kv_lengths(cfg)
+    counts = step_counts(cfg, lengths)
+    b = int(np.argmax(lengths))
+    # one step = the oracle on one head of the longest sequence, extrapolated
+    per = []
+    for i in range(args.warmup + args.steps):
+        t = oracle_sample(cfg, lengths, [i % cfg.H], b)
+        if i >= args.warmup:
+            per.append(t / int(lengths[b]))
+    full_s = statistics.mean(per) * counts["sum_L"] * cfg.H
+    value = counts["step_bytes"] / full_s / 1e12
+    sample = (f"per step: oracle on sequence {b} (L={int(lengths[b])}), 1/{cfg.H} heads; "
+              f"extrapolated per (cached token x head) to {full_s:.4g} s/step")
+    line = {
+        "metric": METRIC, "value": round(value, 8), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(full_s * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, mla_inputs)",
+        "config": {"workload": f"{cfg.name}: B={cfg.B} H={cfg.H} n_q={cfg.n_q} "
+                               f"L={'U[1,%d]' % cfg.L_max if cfg.L is None else cfg.L} d_c=512 d_R=64 d_h=128"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    dist = Dist(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, dist)
+    else:
+        run_ours(args, dist)
+
+
+if __name__ == "__main__":
+    main()

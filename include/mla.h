@@ -1,0 +1,185 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) MLA weight-absorbed decode library.
+ *
+ * Multi-head Latent Attention keeps, per token and layer, only the joint
+ * latent c^KV (d_c = 512) and one RoPE key k^R (d_h^R = 64) shared by all
+ * heads: 576 bf16 elements.  W^UK is folded into each head's query, attention
+ * scores and aggregates directly against the latent cache, and W^UV is
+ * applied after the reduction, so per-head keys and values never exist.
+ *   - "DeepSeek-V2/V3: 大模型的两张账" (chenyuan1125.github.io), section
+ *     "第一张账": c_t^KV = W^DKV h_t, k_t^C = W^UK c_t^KV, v_t^C = W^UV c_t^KV;
+ *     W^UK absorbed into the query side, W^UV applied after aggregating in
+ *     latent space; cache only c_t^KV and k_t^R; (d_c + d_h^R) = 4.5 d_h.
+ *   - DeepSeek-V2 MLA explainer (xinfinite.net), section 2.2.2: decoupled
+ *     RoPE with per-head q^R and one shared k^R; the RoPE'd key part is cached
+ *     so keys need no rotation at inference; attention on [q^C; q^R].[k^C; k^R].
+ *
+ * Fixed sizes: d_c = 512, d_h^R = 64, d_h = 128 (packed cache row D = 576).
+ * Runtime sizes: B sequences, H heads (1..128), n_q new query tokens per
+ * sequence (1..16), T = B * n_q query rows (row t = b * n_q + j).
+ *
+ * Conventions for every entry point:
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory, dense
+ *     row-major, in the layouts stated.  bf16 tensors must be 16-byte aligned.
+ *     The library never allocates, frees, synchronises or keeps a pointer
+ *     after it returns; work is enqueued on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).
+ *   - Host-side argument errors return MLA_ERR_INVALID_ARG or
+ *     MLA_ERR_UNSUPPORTED_SHAPE before anything is launched.  A failed launch
+ *     returns MLA_ERR_CUDA.
+ *   - `dev_status` (nullable) is a device int32 that kernels OR error bits
+ *     into (MLA_DEVERR_*).  The caller zeroes it and reads it after the stream
+ *     is synchronised; mla_device_status_string() names the bits.  Work that
+ *     trips a check is skipped (never a trap or a fault).
+ *   - RoPE pairs adjacent dims (2i, 2i+1) with theta_i = base^(-2i/64); the
+ *     key of cache index t is rotated at position t, query j of sequence b at
+ *     L_b - n_q + j.  `rope_table` is fp32 [rope_len, 64] holding
+ *     (cos, sin) of pos * theta_i for pair i at [pos, 2i], [pos, 2i+1]; build
+ *     it with mla_rope_table_fill() and copy it to the device.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* mla_stream; /* cudaStream_t */
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,       /* null pointer, misalignment, negative size */
+    MLA_ERR_UNSUPPORTED_SHAPE = 2, /* H, n_q or split count outside the supported range */
+    MLA_ERR_CUDA = 3,              /* a CUDA runtime call or launch failed */
+    MLA_ERR_WORKSPACE = 4          /* workspace smaller than the *_workspace_bytes() figure */
+} mla_status;
+
+/* Bits a kernel ORs into *dev_status. */
+#define MLA_DEVERR_ROW_RANGE   0x1  /* a cache row outside [0, cap_tokens) was addressed */
+#define MLA_DEVERR_POS_RANGE   0x2  /* a position outside [0, rope_len) */
+#define MLA_DEVERR_KV_LEN      0x4  /* kv_len[b] < n_q */
+#define MLA_DEVERR_TIMEOUT     0x8  /* a bounded wait in a pipelined kernel expired */
+
+const char* mla_status_string(int status);
+const char* mla_device_status_string(int32_t dev_status_word);
+int mla_abi_version(void);
+
+/*
+ * mla_rope_table_fill -- HOST function.  table_host: fp32 [rope_len, 64],
+ * caller-owned host memory.  Entry [p, 2i] = (float)cos(p * theta_i),
+ * [p, 2i+1] = (float)sin(p * theta_i), theta_i = base^(-2i/64), computed in
+ * double with the C library and rounded once to fp32.
+ */
+mla_status mla_rope_table_fill(float* table_host, int64_t rope_len, double base);
+
+/*
+ * mla_absorb_q -- absorb W^UK into the query and rotate q^R.
+ * (Absorption: "两张账" page, "第一张账" -- W^UK moves to the query side so
+ *  that q^C . k^C_t = q_abs . c_t^KV; decoupled RoPE: explainer 2.2.2.)
+ *   q_nope  bf16 [T, H, 128]     content query q^C
+ *   q_rope  bf16 [T, H, 64]      RoPE query q^R before rotation
+ *   pos     int32 [T] or NULL    position of query row t (NULL: q_rope is
+ *                                already rotated and is copied)
+ *   W_UK    bf16 [H, 128, 512]   per-head up-projection (k^C = W^UK_h c)
+ *   q_out   bf16 [T, H, 576]     [ (W^UK_h)^T q_nope (512) | R_pos q^R (64) ]
+ * fp32 accumulation, one rounding to bf16 per output element.
+ */
+mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* pos,
+                        const void* W_UK, const float* rope_table, int64_t rope_len,
+                        int T, int H, void* q_out, int32_t* dev_status, mla_stream stream);
+
+/*
+ * mla_append_cache -- write T new tokens into the packed latent cache.
+ * ("两张账" page: only c^KV and k^R are cached; explainer 2.2.2: k^R is
+ *  cached already rotated.)
+ *   cache      bf16 [cap_tokens, 576]  row = seq_start[seq_idx[i]] + pos[i]
+ *   seq_start  int64 [*]  first cache row of each sequence
+ *   seq_idx    int32 [T]  sequence of token i
+ *   pos        int32 [T]  position of token i within its sequence
+ *   c_kv       bf16 [T, 512]   copied to columns 0..511 bit for bit
+ *   k_rope     bf16 [T, 64]    rotated at pos[i] into columns 512..575
+ * The rotation is y0 = fl(fl(x0 c) - fl(x1 s)), y1 = fl(fl(x0 s) + fl(x1 c))
+ * in fp32 (no fused multiply-add) with (c, s) from rope_table, then
+ * round-to-nearest-even to bf16: the result is reproducible bit for bit.
+ * Out-of-range rows or positions set a MLA_DEVERR_* bit and are skipped.
+ */
+mla_status mla_append_cache(void* cache, int64_t cap_tokens, const int64_t* seq_start,
+                            const int32_t* seq_idx, const int32_t* pos, const void* c_kv,
+                            const void* k_rope, const float* rope_table, int64_t rope_len,
+                            int T, int32_t* dev_status, mla_stream stream);
+
+/*
+ * mla_decode_workspace_bytes -- device workspace mla_decode needs for these
+ * sizes (num_splits as passed to mla_decode; 0 = automatic).
+ */
+size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
+
+/*
+ * mla_decode -- one absorbed MLA decode step over the latent cache.
+ * For every sequence b, query j and head h, with p = kv_len[b] - n_q + j:
+ *   s_t   = (q[t,h,:512] . c_t + q[t,h,512:] . k^R_t) * scale,  t = 0..p
+ *   P     = softmax(s)                   (fp32, online / split-KV)
+ *   o_lat = sum_t P_t c_t                (latent aggregation, 512)
+ *   out   = W^UV_h o_lat                 (128)
+ * ("两张账" page, "第一张账": scores against the cached latent, aggregation in
+ *  latent space, W^UV afterwards; explainer 2.2.2 for the concatenated
+ *  content/position inner product.)
+ *   q          bf16 [B*n_q, H, 576]   from mla_absorb_q
+ *   cache      bf16 [cap_tokens, 576] sequence b occupies rows
+ *              seq_start[b] .. seq_start[b] + kv_len[b] - 1 (kv_len counts
+ *              the n_q tokens of this step, already appended)
+ *   seq_start  int64 [B];  kv_len int32 [B]
+ *   W_UV       bf16 [H, 128, 512]
+ *   scale      softmax scale, 1/sqrt(d_h + d_h^R) = 1/sqrt(192) for V2 shapes
+ *   num_splits KV splits per sequence for the partial/merge path (0 = automatic)
+ *   workspace  device scratch of at least mla_decode_workspace_bytes() bytes
+ *   out        bf16 [B*n_q, H, 128]
+ *   lse_out    fp32 [B*n_q, H] or NULL: log sum_t exp(s_t)
+ * A sequence with kv_len[b] < n_q sets MLA_DEVERR_KV_LEN and its rows are
+ * left unwritten; rows beyond cap_tokens set MLA_DEVERR_ROW_RANGE.
+ */
+mla_status mla_decode(const void* q, const void* cache, int64_t cap_tokens,
+                      const int64_t* seq_start, const int32_t* kv_len, const void* W_UV,
+                      int B, int n_q, int H, float scale, int num_splits,
+                      void* workspace, size_t ws_bytes, void* out, float* lse_out,
+                      int32_t* dev_status, mla_stream stream);
+
+/*
+ * mla_decode_attend / mla_decode_finish -- the two phases of mla_decode,
+ * exposed so that callers can place work (or timing events) between them.
+ * attend: scores, online softmax and latent aggregation into per-split
+ * partials held in `workspace`; finish: log-sum-exp merge of the partials
+ * and the W^UV up-projection into `out` (and `lse_out`).  Arguments mean the
+ * same as for mla_decode; both calls must see the same sizes, num_splits and
+ * workspace, and finish must be ordered after attend on the stream.
+ */
+mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_tokens,
+                             const int64_t* seq_start, const int32_t* kv_len,
+                             int B, int n_q, int H, float scale, int num_splits,
+                             void* workspace, size_t ws_bytes, int32_t* dev_status,
+                             mla_stream stream);
+mla_status mla_decode_finish(const void* W_UV, int B, int n_q, int H, int num_splits,
+                             void* workspace, size_t ws_bytes, void* out, float* lse_out,
+                             mla_stream stream);
+
+/*
+ * mla_splitkv_combine -- log-sum-exp merge of split-KV partials.
+ *   o_part   fp32 [T, H, S, 512]  each split's softmax-normalised latent output
+ *   lse_part fp32 [T, H, S]       each split's log-sum-exp (-inf: empty split)
+ * m = max_s lse_s, w_s = exp(lse_s - m): o = sum_s w_s o_s / sum_s w_s and
+ * lse = m + log sum_s w_s.  With W_UV (bf16 [H,128,512]) the merged latent
+ * is mapped out: out bf16 [T, H, 128]; with W_UV == NULL, out is the merged
+ * latent, fp32 [T, H, 512].  lse_out fp32 [T, H] or NULL.
+ */
+mla_status mla_splitkv_combine(const float* o_part, const float* lse_part, int T, int H,
+                               int num_splits, const void* W_UV, void* out, float* lse_out,
+                               mla_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */

@@ -1,0 +1,169 @@
+// extern "C" entry points of libmla_b200: host-side validation, workspace
+// layout and kernel launches.  Every function is asynchronous on the caller's
+// stream; nothing here allocates, synchronises or keeps pointers.
+#include <math.h>
+#include <stdint.h>
+
+#include "mla_internal.cuh"
+
+namespace {
+
+using namespace mla;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int auto_splits(int B, int n_q, int H) {
+    const int rowblocks = (n_q * H + 15) / 16;
+    const int ctas = B * rowblocks;
+    int s = (2 * 148 + ctas - 1) / ctas;
+    return s < 1 ? 1 : (s > 64 ? 64 : s);
+}
+
+struct DecodeWs {
+    size_t o_part, lse_part, total;
+};
+
+DecodeWs decode_ws_layout(int B, int n_q, int H, int S) {
+    const size_t rows = static_cast<size_t>(B) * n_q * H;
+    DecodeWs w;
+    w.o_part = 0;
+    w.lse_part = rows * S * kDc * sizeof(float);
+    w.total = w.lse_part + ((rows * S * sizeof(float) + 255) / 256) * 256;
+    return w;
+}
+
+mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int mla_abi_version(void) { return 1; }
+
+const char* mla_status_string(int status) {
+    switch (status) {
+        case MLA_OK: return "ok";
+        case MLA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, negative size)";
+        case MLA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (H in 1..128, n_q in 1..16, splits in 0..256)";
+        case MLA_ERR_CUDA: return "CUDA runtime error";
+        case MLA_ERR_WORKSPACE: return "workspace too small";
+        default: return "unknown status";
+    }
+}
+
+const char* mla_device_status_string(int32_t w) {
+    if (w == 0) return "ok";
+    if (w & MLA_DEVERR_TIMEOUT) return "bounded wait expired in a pipelined kernel";
+    if (w & MLA_DEVERR_ROW_RANGE) return "cache row outside [0, cap_tokens)";
+    if (w & MLA_DEVERR_POS_RANGE) return "position outside the RoPE table";
+    if (w & MLA_DEVERR_KV_LEN) return "kv_len smaller than n_q";
+    return "unknown device error bits";
+}
+
+mla_status mla_rope_table_fill(float* table, int64_t rope_len, double base) {
+    if (!table || rope_len < 0 || !(base > 0.0)) return MLA_ERR_INVALID_ARG;
+    double theta[kDr / 2];
+    for (int i = 0; i < kDr / 2; ++i) theta[i] = pow(base, -2.0 * i / (double)kDr);
+    for (int64_t p = 0; p < rope_len; ++p) {
+        for (int i = 0; i < kDr / 2; ++i) {
+            const double ang = (double)p * theta[i];
+            table[p * kDr + 2 * i] = (float)cos(ang);
+            table[p * kDr + 2 * i + 1] = (float)sin(ang);
+        }
+    }
+    return MLA_OK;
+}
+
+mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* pos, const void* W_UK,
+                        const float* rope_table, int64_t rope_len, int T, int H, void* q_out,
+                        int32_t* dev_status, mla_stream stream) {
+    if (T < 0 || rope_len < 0) return MLA_ERR_INVALID_ARG;
+    if (H < 1 || H > kMaxHeads) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MLA_OK;
+    if (!q_nope || !q_rope || !W_UK || !q_out || (pos && !rope_table)) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(W_UK) || !aligned16(q_out)) return MLA_ERR_INVALID_ARG;
+    return cuda_status(launch_absorb_q(static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_rope),
+                                       pos, static_cast<const uint16_t*>(W_UK), rope_table, rope_len, T, H,
+                                       static_cast<uint16_t*>(q_out), dev_status,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_append_cache(void* cache, int64_t cap_tokens, const int64_t* seq_start, const int32_t* seq_idx,
+                            const int32_t* pos, const void* c_kv, const void* k_rope, const float* rope_table,
+                            int64_t rope_len, int T, int32_t* dev_status, mla_stream stream) {
+    if (T < 0 || cap_tokens < 0 || rope_len < 0) return MLA_ERR_INVALID_ARG;
+    if (T == 0) return MLA_OK;
+    if (!cache || !seq_start || !seq_idx || !pos || !c_kv || !k_rope || !rope_table) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(cache) || !aligned16(c_kv) || !aligned16(k_rope) || !aligned16(rope_table))
+        return MLA_ERR_INVALID_ARG;
+    return cuda_status(launch_append_cache(static_cast<uint16_t*>(cache), cap_tokens, seq_start, seq_idx, pos,
+                                           static_cast<const uint16_t*>(c_kv), static_cast<const uint16_t*>(k_rope),
+                                           rope_table, rope_len, T, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits) {
+    if (B < 0 || n_q < 1 || H < 1 || num_splits < 0) return 0;
+    const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
+    return decode_ws_layout(B, n_q, H, S).total;
+}
+
+mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_tokens, const int64_t* seq_start,
+                             const int32_t* kv_len, int B, int n_q, int H, float scale, int num_splits,
+                             void* workspace, size_t ws_bytes, int32_t* dev_status, mla_stream stream) {
+    if (B < 0 || cap_tokens < 0 || !(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
+    if (H < 1 || H > kMaxHeads || n_q < 1 || n_q > kMaxNq || num_splits < 0 || num_splits > 256)
+        return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0) return MLA_OK;
+    if (!q || !cache || !seq_start || !kv_len || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(cache) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
+    const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
+    const DecodeWs lay = decode_ws_layout(B, n_q, H, S);
+    if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
+    float* o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.o_part);
+    float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.lse_part);
+    return cuda_status(launch_decode_simt(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(cache),
+                                          cap_tokens, seq_start, kv_len, B, n_q, H, scale, S, o_part, lse_part,
+                                          dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_decode_finish(const void* W_UV, int B, int n_q, int H, int num_splits, void* workspace,
+                             size_t ws_bytes, void* out, float* lse_out, mla_stream stream) {
+    if (B < 0) return MLA_ERR_INVALID_ARG;
+    if (H < 1 || H > kMaxHeads || n_q < 1 || n_q > kMaxNq || num_splits < 0 || num_splits > 256)
+        return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0) return MLA_OK;
+    if (!W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(W_UV) || !aligned16(out) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
+    const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
+    const DecodeWs lay = decode_ws_layout(B, n_q, H, S);
+    if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
+    const float* o_part = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + lay.o_part);
+    const float* lse_part = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + lay.lse_part);
+    return cuda_status(launch_combine(o_part, lse_part, B * n_q, H, S, static_cast<const uint16_t*>(W_UV), out,
+                                      lse_out, static_cast<cudaStream_t>(stream)));
+}
+
+mla_status mla_decode(const void* q, const void* cache, int64_t cap_tokens, const int64_t* seq_start,
+                      const int32_t* kv_len, const void* W_UV, int B, int n_q, int H, float scale, int num_splits,
+                      void* workspace, size_t ws_bytes, void* out, float* lse_out, int32_t* dev_status,
+                      mla_stream stream) {
+    if (B > 0 && (!W_UV || !out)) return MLA_ERR_INVALID_ARG;
+    if (B > 0 && (!aligned16(W_UV) || !aligned16(out))) return MLA_ERR_INVALID_ARG;
+    mla_status st = mla_decode_attend(q, cache, cap_tokens, seq_start, kv_len, B, n_q, H, scale, num_splits,
+                                      workspace, ws_bytes, dev_status, stream);
+    if (st != MLA_OK || B == 0) return st;
+    return mla_decode_finish(W_UV, B, n_q, H, num_splits, workspace, ws_bytes, out, lse_out, stream);
+}
+
+mla_status mla_splitkv_combine(const float* o_part, const float* lse_part, int T, int H, int num_splits,
+                               const void* W_UV, void* out, float* lse_out, mla_stream stream) {
+    if (T < 0) return MLA_ERR_INVALID_ARG;
+    if (H < 1 || H > kMaxHeads || num_splits < 1 || num_splits > 256) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MLA_OK;
+    if (!o_part || !lse_part || !out) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(o_part) || !aligned16(out) || (W_UV && !aligned16(W_UV))) return MLA_ERR_INVALID_ARG;
+    return cuda_status(launch_combine(o_part, lse_part, T, H, num_splits, static_cast<const uint16_t*>(W_UV), out,
+                                      lse_out, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

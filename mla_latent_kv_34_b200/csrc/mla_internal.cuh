@@ -1,0 +1,56 @@
+// Internal helpers shared by the MLA kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+constexpr int kDc = 512;           // latent width d_c
+constexpr int kDr = 64;            // RoPE width d_h^R
+constexpr int kDh = 128;           // head width d_h
+constexpr int kRow = kDc + kDr;    // packed cache row (576 bf16 = 1152 B)
+constexpr int kMaxHeads = 128;
+constexpr int kMaxNq = 16;
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// fp32 -> bf16, round to nearest, ties to even (finite inputs; NaN kept quiet).
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return static_cast<uint16_t>((u >> 16) | 0x40u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return static_cast<uint16_t>(u >> 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    return static_cast<uint32_t>(f32_to_bf16_rne(lo)) | (static_cast<uint32_t>(f32_to_bf16_rne(hi)) << 16);
+}
+
+__device__ __forceinline__ void report(int32_t* dev_status, int32_t bit) {
+    if (dev_status) atomicOr(dev_status, bit);
+}
+
+// Host-side launch wrappers (one per kernel file).
+cudaError_t launch_append_cache(uint16_t* cache, int64_t cap, const int64_t* seq_start, const int32_t* seq_idx,
+                                const int32_t* pos, const uint16_t* c_kv, const uint16_t* k_rope,
+                                const float* rope_table, int64_t rope_len, int T, int32_t* dev_status,
+                                cudaStream_t stream);
+
+cudaError_t launch_absorb_q(const uint16_t* q_nope, const uint16_t* q_rope, const int32_t* pos,
+                            const uint16_t* W_UK, const float* rope_table, int64_t rope_len, int T, int H,
+                            uint16_t* q_out, int32_t* dev_status, cudaStream_t stream);
+
+cudaError_t launch_decode_simt(const uint16_t* q, const uint16_t* cache, int64_t cap, const int64_t* seq_start,
+                               const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,
+                               float* o_part, float* lse_part, int32_t* dev_status, cudaStream_t stream);
+
+cudaError_t launch_combine(const float* o_part, const float* lse_part, int T, int H, int splits,
+                           const uint16_t* W_UV, void* out, float* lse_out, cudaStream_t stream);
+
+}  // namespace mla

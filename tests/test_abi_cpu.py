@@ -1,0 +1,87 @@
+"""The C-ABI library on the CPU: it loads, exports every declared symbol, its
+host-side table matches the oracle's bit for bit, and host validation rejects
+bad arguments before any CUDA call (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+@pytest.fixture(scope="module")
+def mla():
+    import mla_latent_kv_34_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(mla):
+    names = declared_functions()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(mla.lib, n), n
+    assert set(names) == set(mla.EXPORTED)
+    assert mla.lib.mla_abi_version() == 1
+
+
+def test_rope_table_matches_oracle_bitwise(mla):
+    from oracle.append import rope_table_f32
+    n = 3000
+    host = np.empty((n, 64), dtype=np.float32)
+    assert mla.lib.mla_rope_table_fill(host.ctypes.data_as(ctypes.c_void_p), n, 10000.0) == 0
+    pos = list(range(0, n, 7)) + [n - 1]
+    c, s = rope_table_f32(pos)
+    np.testing.assert_array_equal(host[pos][:, 0::2], c)
+    np.testing.assert_array_equal(host[pos][:, 1::2], s)
+
+
+def test_status_strings(mla):
+    assert mla.lib.mla_status_string(0) == b"ok"
+    assert b"workspace" in mla.lib.mla_status_string(4)
+    assert b"kv_len" in mla.lib.mla_device_status_string(4)
+    assert mla.lib.mla_device_status_string(0) == b"ok"
+
+
+def test_host_validation_rejects_bad_arguments(mla):
+    L = mla.lib
+    fake = ctypes.c_void_p(4096)  # never dereferenced: validation fails first
+    odd = ctypes.c_void_p(4098)
+    # decode: null q, unsupported H / n_q / splits, bad scale, small workspace
+    assert L.mla_decode(None, fake, 10, fake, fake, fake, 1, 1, 16, 0.07, 0, fake, 1 << 30, fake, None, None, None) == 1
+    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 1, 1, 129, 0.07, 0, fake, 1 << 30, fake, None, None, None) == 2
+    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 1, 0, 16, 0.07, 0, fake, 1 << 30, fake, None, None, None) == 2
+    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 1, 1, 16, 0.07, 300, fake, 1 << 30, fake, None, None, None) == 2
+    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 1, 1, 16, -1.0, 0, fake, 1 << 30, fake, None, None, None) == 1
+    assert L.mla_decode(odd, fake, 10, fake, fake, fake, 1, 1, 16, 0.07, 0, fake, 1 << 30, fake, None, None, None) == 1
+    need = L.mla_decode_workspace_bytes(4, 2, 128, 3)
+    assert need > 0
+    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 4, 2, 128, 0.07, 3, fake, need - 1, fake, None, None,
+                        None) == 4
+    # empty batch is a no-op
+    assert L.mla_decode(None, None, 0, None, None, None, 0, 1, 16, 0.07, 0, None, 0, None, None, None, None) == 0
+    # absorb / append / combine
+    assert L.mla_absorb_q(fake, fake, None, fake, None, 0, 4, 0, fake, None, None) == 2
+    assert L.mla_absorb_q(None, fake, None, fake, None, 0, 4, 16, fake, None, None) == 1
+    assert L.mla_absorb_q(None, None, None, None, None, 0, 0, 16, None, None, None) == 0
+    assert L.mla_append_cache(fake, 10, fake, fake, fake, fake, fake, None, 5, 3, None, None) == 1
+    assert L.mla_append_cache(fake, -1, fake, fake, fake, fake, fake, fake, 5, 3, None, None) == 1
+    assert L.mla_append_cache(None, 0, None, None, None, None, None, None, 0, 0, None, None) == 0
+    assert L.mla_splitkv_combine(fake, fake, 4, 16, 0, None, fake, None, None) == 2
+    assert L.mla_splitkv_combine(None, fake, 4, 16, 2, None, fake, None, None) == 1
+
+
+def test_workspace_grows_with_splits(mla):
+    a = mla.decode_workspace_bytes(32, 1, 128, 1)
+    b = mla.decode_workspace_bytes(32, 1, 128, 4)
+    assert b > a > 0
+    assert mla.decode_workspace_bytes(32, 1, 128, 0) > 0

@@ -1,0 +1,252 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Tolerance (stated for the decode output): |gpu - ref| <= 1e-2 + 1e-2 |ref| per
+element, with bf16 inputs and fp32 accumulation; in addition the relative L2
+error over the compared block must stay below 1e-2 and lse within 2e-2
+(absolute, natural-log units).  The append is compared bit for bit.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mla_inputs as mi
+from oracle import append as oapp
+from oracle import naive as on
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 1e-2, 1e-2
+
+
+@pytest.fixture(scope="module")
+def H():
+    import gpu_harness
+    return gpu_harness
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _check_decode(prob, out, lse, seqs, heads=None, label=""):
+    from gpu_harness import rel_l2, tol_excess
+    cfg = prob.cfg
+    got_all = out.float().cpu().numpy().reshape(cfg.B, cfg.n_q, cfg.H, mi.D_H)
+    lse_all = lse.cpu().numpy().reshape(cfg.B, cfg.n_q, cfg.H)
+    hs = list(range(cfg.H)) if heads is None else list(heads)
+    for b in seqs:
+        ref, _, ref_lse = prob.oracle(b, heads=hs)
+        got = got_all[b][:, hs]
+        ex = tol_excess(got, ref, ATOL, RTOL)
+        assert ex <= 0, f"{label} seq {b} (L={prob.lengths[b]}): tolerance exceeded by {ex:.3e}"
+        assert rel_l2(got, ref) < 1e-2, f"{label} seq {b}: rel L2 {rel_l2(got, ref):.3e}"
+        assert np.abs(lse_all[b][:, hs] - ref_lse).max() < 2e-2, f"{label} seq {b}: lse"
+        assert np.all(np.isfinite(got))
+
+
+# ----------------------------------------------------------------- append
+
+def test_append_bit_exact_with_canary(cuda_ok, H):
+    dev = "cuda"
+    import mla_latent_kv_34_b200 as mla
+    cap = 5000
+    canary = np.full((cap, 576), 0xA5A5, dtype=np.uint16)
+    cache = H.to_dev_bf16(canary, dev)
+    starts = np.array([0, 1000, 2500, 4000], dtype=np.int64)
+    rng = np.random.default_rng(1)
+    T = 777
+    seq_idx = rng.integers(0, 4, T).astype(np.int32)
+    # distinct positions per sequence so no row is written twice
+    pos = np.empty(T, dtype=np.int32)
+    for s in range(4):
+        idx = np.where(seq_idx == s)[0]
+        pos[idx] = rng.choice(900, len(idx), replace=False)
+    c = mi.normal_bf16(77, 1, 0, T * 512).reshape(T, 512)
+    k = mi.normal_bf16(77, 2, 0, T * 64).reshape(T, 64)
+    tab = mla.rope_table(1000, 10000.0, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    mla.append_cache(cache, torch.from_numpy(starts).to(dev), torch.from_numpy(seq_idx).to(dev),
+                     torch.from_numpy(pos).to(dev), H.to_dev_bf16(c, dev), H.to_dev_bf16(k, dev), tab, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = oapp.append_rows(canary, starts, seq_idx, pos, c, k)
+    np.testing.assert_array_equal(_bits(cache), ref)
+
+
+def test_append_large_positions_bit_exact(cuda_ok, H):
+    import mla_latent_kv_34_b200 as mla
+    dev = "cuda"
+    T = 512
+    pos = (np.arange(T, dtype=np.int64) * 257 + 131071 - 257 * 511).astype(np.int32)
+    cap = int(pos.max()) + 1
+    cache = torch.zeros((cap, 576), dtype=torch.bfloat16, device=dev)
+    c = mi.normal_bf16(78, 1, 0, T * 512).reshape(T, 512)
+    k = mi.normal_bf16(78, 2, 0, T * 64).reshape(T, 64)
+    tab = mla.rope_table(131072, 10000.0, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    mla.append_cache(cache, torch.zeros(1, dtype=torch.int64, device=dev), torch.zeros(T, dtype=torch.int32, device=dev),
+                     torch.from_numpy(pos).to(dev), H.to_dev_bf16(c, dev), H.to_dev_bf16(k, dev), tab, st)
+    got = _bits(cache[torch.from_numpy(pos.astype(np.int64)).to(dev)])
+    np.testing.assert_array_equal(got[:, :512], c)
+    np.testing.assert_array_equal(got[:, 512:], oapp.rotate_k_bits(k, pos))
+    assert int(st.item()) == 0
+
+
+def test_append_out_of_range_is_reported_and_skipped(cuda_ok, H):
+    import mla_latent_kv_34_b200 as mla
+    dev = "cuda"
+    cache = torch.zeros((10, 576), dtype=torch.bfloat16, device=dev)
+    tab = mla.rope_table(64, 10000.0, dev)
+    c = torch.ones((2, 512), dtype=torch.bfloat16, device=dev)
+    k = torch.ones((2, 64), dtype=torch.bfloat16, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    mla.append_cache(cache, torch.tensor([0, 8], device=dev), torch.tensor([0, 1], dtype=torch.int32, device=dev),
+                     torch.tensor([3, 5], dtype=torch.int32, device=dev), c, k, tab, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 0x1
+    assert cache[3].float().sum().item() != 0 and cache[9].float().abs().sum().item() == 0
+    st.zero_()
+    mla.append_cache(cache, torch.tensor([0], device=dev), torch.tensor([0], dtype=torch.int32, device=dev),
+                     torch.tensor([9], dtype=torch.int32, device=dev), c[:1], k[:1], tab[:5], st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 0x2
+
+
+# ----------------------------------------------------------------- absorb
+
+@pytest.mark.parametrize("T,Hh", [(1, 16), (37, 16), (32, 128), (256, 128), (5, 3)])
+def test_absorb_q_matches_oracle(cuda_ok, H, T, Hh):
+    import mla_latent_kv_34_b200 as mla
+    dev = "cuda"
+    cfg = mi.MLAConfig("absorb", B=T, H=Hh, n_q=1, L=10, seed=900 + T)
+    qn, qr = mi.queries(cfg)
+    Wk = mi.weights(cfg, "uk")
+    pos = ((np.arange(T) * 7919) % 131072).astype(np.int32)
+    tab = mla.rope_table(131072, 10000.0, dev)
+    q = mla.absorb_q(H.to_dev_bf16(qn, dev), H.to_dev_bf16(qr, dev), torch.from_numpy(pos).to(dev),
+                     H.to_dev_bf16(Wk, dev), tab)
+    got = q.float().cpu().numpy()
+    f = mi.bf16_bits_to_f64
+    ref_abs = on.absorb_query(f(qn), f(Wk))
+    ref_pe = on.rope(f(qr), pos[:, None])
+    # one bf16 rounding of an fp32-accumulated value: relative 2^-8 plus tiny absolute
+    assert np.all(np.abs(got[..., :512] - ref_abs) <= 1e-3 + 2 ** -8 * np.abs(ref_abs))
+    assert np.all(np.abs(got[..., 512:] - ref_pe) <= 1e-6 + 2 ** -7 * np.abs(ref_pe))
+    # rope part is bit-identical to the append arithmetic
+    exp_bits = oapp.rotate_k_bits(qr.reshape(-1, 64), np.repeat(pos, Hh)).reshape(T, Hh, 64)
+    np.testing.assert_array_equal(_bits(q)[..., 512:], exp_bits)
+    # pos = NULL copies q^R as given
+    q2 = mla.absorb_q(H.to_dev_bf16(qn, dev), H.to_dev_bf16(qr, dev), None, H.to_dev_bf16(Wk, dev), tab)
+    np.testing.assert_array_equal(_bits(q2)[..., 512:], qr)
+
+
+# ----------------------------------------------------------------- decode
+
+def test_decode_tiny_full(cuda_ok, H):
+    prob = H.build_problem(mi.CONFIGS["tiny"])
+    out, lse = prob.decode(prob.absorb())
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    _check_decode(prob, out, lse, [0], label="tiny")
+
+
+@pytest.mark.parametrize("L,n_q,Hh", [(1, 1, 16), (2, 2, 16), (3, 2, 128), (64, 1, 128), (65, 2, 128),
+                                      (127, 1, 1), (200, 2, 100), (1000, 1, 64), (129, 2, 64)])
+def test_decode_edge_shapes(cuda_ok, H, L, n_q, Hh):
+    cfg = mi.MLAConfig("edge", B=2, H=Hh, n_q=n_q, L=L, seed=1000 + L + Hh)
+    prob = H.build_problem(cfg, lengths=[L, max(n_q, L // 2 + 1)])
+    out, lse = prob.decode(prob.absorb())
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    _check_decode(prob, out, lse, [0, 1], label=f"edge L={L}")
+
+
+def test_decode_small_ragged_full(cuda_ok, H):
+    cfg = mi.MLAConfig("ragged-small", B=12, H=128, n_q=2, L=None, L_max=700, seed=77)
+    prob = H.build_problem(cfg)
+    out, lse = prob.decode(prob.absorb())
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    _check_decode(prob, out, lse, range(cfg.B), heads=range(0, 128, 5), label="ragged-small")
+
+
+@pytest.mark.parametrize("splits", [1, 2, 7, 32])
+def test_decode_split_invariance(cuda_ok, H, splits):
+    cfg = mi.MLAConfig("splits", B=3, H=32, n_q=2, L=None, L_max=3000, seed=55)
+    prob = H.build_problem(cfg)
+    q = prob.absorb()
+    ref_out, ref_lse = prob.decode(q, num_splits=1)
+    out, lse = prob.decode(q, num_splits=splits)
+    torch.cuda.synchronize()
+    a, b = out.float().cpu().numpy(), ref_out.float().cpu().numpy()
+    # same math up to fp32 summation order, then one bf16 rounding
+    assert np.all(np.abs(a - b) <= 1e-4 + 2 ** -7 * np.abs(b))
+    assert np.abs(lse.cpu().numpy() - ref_lse.cpu().numpy()).max() < 1e-4
+    _check_decode(prob, out, lse, [0, 2], label=f"splits={splits}")
+
+
+@pytest.mark.parametrize("name,seqs,heads", [
+    ("v2lite", [0, 63], None),
+    ("v2", [0, 31], range(0, 128, 9)),
+    ("128k", [3], range(0, 128, 31)),
+])
+def test_decode_full_size_sampled(cuda_ok, H, name, seqs, heads):
+    cfg = mi.CONFIGS[name]
+    prob = H.build_problem(cfg)
+    out, lse = prob.decode(prob.absorb())
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    _check_decode(prob, out, lse, seqs, heads=heads, label=name)
+    # every row finite, lse >= log(1)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_decode_ragged_full_size_sampled(cuda_ok, H):
+    cfg = mi.CONFIGS["ragged"]
+    prob = H.build_problem(cfg)
+    out, lse = prob.decode(prob.absorb())
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    L = prob.lengths
+    pick = sorted({int(np.argmin(L)), int(np.argmax(L)), 0, 77})
+    _check_decode(prob, out, lse, pick, heads=range(0, 128, 16), label="ragged")
+    assert torch.isfinite(out.float()).all()
+
+
+def test_decode_reports_short_kv_len(cuda_ok, H):
+    cfg = mi.MLAConfig("short", B=2, H=16, n_q=2, L=10, seed=3)
+    prob = H.build_problem(cfg)
+    prob.kv_len[1] = 1
+    prob.decode(prob.absorb())
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) & 0x4
+
+
+# ----------------------------------------------------------------- combine
+
+@pytest.mark.parametrize("with_wuv", [False, True])
+def test_splitkv_combine_matches_oracle_merge(cuda_ok, H, with_wuv):
+    import mla_latent_kv_34_b200 as mla
+    dev = "cuda"
+    T, Hh, S = 5, 8, 6
+    rng = np.random.default_rng(4)
+    o = rng.standard_normal((T, Hh, S, 512)).astype(np.float32)
+    lse = (rng.standard_normal((T, Hh, S)) * 3).astype(np.float32)
+    lse[0, 0, :] = -np.inf
+    lse[0, 0, 2] = 1.5          # one live split
+    lse[1, 1, 3:] = -np.inf     # empty splits
+    Wv = mi.normal_bf16(9, 6, 0, Hh * 128 * 512, 1 / math.sqrt(512)).reshape(Hh, 128, 512)
+    lse_out = torch.empty((T, Hh), dtype=torch.float32, device=dev)
+    out = mla.splitkv_combine(torch.from_numpy(o).to(dev), torch.from_numpy(lse).to(dev),
+                              W_UV=H.to_dev_bf16(Wv, dev) if with_wuv else None, lse_out=lse_out)
+    ref_o, ref_lse = on.merge_partials(np.moveaxis(o, 2, 0).astype(np.float64), np.moveaxis(lse, 2, 0))
+    np.testing.assert_allclose(lse_out.cpu().numpy(), ref_lse, rtol=1e-5, atol=1e-5)
+    if with_wuv:
+        ref = on.up_project(ref_o, mi.bf16_bits_to_f64(Wv))
+        got = out.float().cpu().numpy()
+        assert np.all(np.abs(got - ref) <= 1e-3 + 2 ** -7 * np.abs(ref))
+    else:
+        np.testing.assert_allclose(out.cpu().numpy(), ref_o, rtol=1e-5, atol=1e-6)
