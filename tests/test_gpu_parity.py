@@ -80,7 +80,7 @@ def test_append_large_positions_bit_exact(cuda_ok, H):
     import mla_latent_kv_34_b200 as mla
     dev = "cuda"
     T = 512
-    pos = (np.arange(T, dtype=np.int64) * 257 + 131071 - 257 * 511).astype(np.int32)
+    pos = (131071 - 255 * (T - 1 - np.arange(T, dtype=np.int64))).astype(np.int32)
     cap = int(pos.max()) + 1
     cache = torch.zeros((cap, 576), dtype=torch.bfloat16, device=dev)
     c = mi.normal_bf16(78, 1, 0, T * 512).reshape(T, 512)
