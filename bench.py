@@ -42,7 +42,7 @@ UNIT = "TB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # kernels each C-ABI call of the step launches
 KERNELS_PER_STEP = {"append": 1, "absorb": 1, "attend": 1, "finish": 1}
-CORE_SOURCES = ["mla_latent_kv_34_b200/csrc/decode_simt.cu"]
+CORE_SOURCES = ["mla_latent_kv_34_b200/csrc/decode_tc.cu", "mla_latent_kv_34_b200/csrc/sm100.cuh"]
 
 
 def parse_args():
@@ -272,7 +272,7 @@ def run_step(mla, cfg, st, ev=None):
                       dev_status=st["status"])
     if ev:
         ev[2].record()
-    mla.decode_finish(st["W_UV"], cfg.B, cfg.n_q, 0, st["ws"], st["out"])
+    mla.decode_finish(st["seq_start"], st["kv_len"], st["cache"], st["W_UV"], cfg.n_q, 0, st["ws"], st["out"])
     if ev:
         ev[3].record()
 

@@ -134,7 +134,11 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
  *   seq_start  int64 [B];  kv_len int32 [B]
  *   W_UV       bf16 [H, 128, 512]
  *   scale      softmax scale, 1/sqrt(d_h + d_h^R) = 1/sqrt(192) for V2 shapes
- *   num_splits KV splits per sequence for the partial/merge path (0 = automatic)
+ *   num_splits 0: use every SM.  n > 0: at most n CTA pairs per group of 128
+ *              query rows.  The (sequence, 64-token tile) space is cut into
+ *              equal contiguous ranges, one per CTA pair; the pieces of a
+ *              sequence are merged by log-sum-exp.  Results do not depend on
+ *              n beyond fp32 summation order.
  *   workspace  device scratch of at least mla_decode_workspace_bytes() bytes
  *   out        bf16 [B*n_q, H, 128]
  *   lse_out    fp32 [B*n_q, H] or NULL: log sum_t exp(s_t)
@@ -161,9 +165,25 @@ mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_token
                              int B, int n_q, int H, float scale, int num_splits,
                              void* workspace, size_t ws_bytes, int32_t* dev_status,
                              mla_stream stream);
-mla_status mla_decode_finish(const void* W_UV, int B, int n_q, int H, int num_splits,
+mla_status mla_decode_finish(const int64_t* seq_start, const int32_t* kv_len, int64_t cap_tokens,
+                             const void* W_UV, int B, int n_q, int H, int num_splits,
                              void* workspace, size_t ws_bytes, void* out, float* lse_out,
                              mla_stream stream);
+
+/*
+ * mla_decode_cudacore -- the same decode step computed on CUDA cores (fp32
+ * FMA, split-KV over `num_splits` equal key ranges per sequence, 0 =
+ * automatic) instead of the tensor cores.  Same arguments and results as
+ * mla_decode, within fp32 rounding; a second implementation to check the
+ * tensor-core path against.  Its workspace size is
+ * mla_decode_cudacore_workspace_bytes().
+ */
+size_t mla_decode_cudacore_workspace_bytes(int B, int n_q, int H, int num_splits);
+mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_tokens,
+                               const int64_t* seq_start, const int32_t* kv_len, const void* W_UV,
+                               int B, int n_q, int H, float scale, int num_splits,
+                               void* workspace, size_t ws_bytes, void* out, float* lse_out,
+                               int32_t* dev_status, mla_stream stream);
 
 /*
  * mla_splitkv_combine -- log-sum-exp merge of split-KV partials.

@@ -36,7 +36,10 @@ _SIGS = {
     "mla_decode_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
     "mla_decode": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
     "mla_decode_attend": ([_p, _p, _i64, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p], _i32),
-    "mla_decode_finish": ([_p, _i32, _i32, _i32, _i32, _p, _sz, _p, _p, _p], _i32),
+    "mla_decode_finish": ([_p, _p, _i64, _p, _i32, _i32, _i32, _i32, _p, _sz, _p, _p, _p], _i32),
+    "mla_decode_cudacore_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
+    "mla_decode_cudacore": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p],
+                            _i32),
     "mla_splitkv_combine": ([_p, _p, _i32, _i32, _i32, _p, _p, _p, _p], _i32),
 }
 for _name, (_args, _ret) in _SIGS.items():
@@ -152,14 +155,39 @@ def decode_attend(q, cache, seq_start, kv_len, n_q: int, scale: float, num_split
         _stream(stream)))
 
 
-def decode_finish(W_UV, B: int, n_q: int, num_splits: int, workspace, out, lse_out=None, stream=None):
+def decode_finish(seq_start, kv_len, cache, W_UV, n_q: int, num_splits: int, workspace, out, lse_out=None,
+                  stream=None):
     """Phase 2 of decode: merge the partials, apply W^UV into ``out`` bf16 [B*n_q, H, 128]."""
+    B = kv_len.shape[0]
     H = W_UV.shape[0]
     _check(lib.mla_decode_finish(
+        _ptr(seq_start, torch.int64, (B,), "seq_start"), _ptr(kv_len, torch.int32, (B,), "kv_len"), cache.shape[0],
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(out, torch.bfloat16, (B * n_q, H, D_H), "out"), _ptr(lse_out, torch.float32, (B * n_q, H), "lse_out"),
         _stream(stream)))
+    return out
+
+
+def decode_cudacore(q, cache, seq_start, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
+                    workspace=None, out=None, lse_out=None, dev_status=None, stream=None):
+    """The decode step on CUDA cores (second implementation, same results within fp32 rounding)."""
+    B = kv_len.shape[0]
+    T, H = q.shape[0], q.shape[1]
+    if T != B * n_q:
+        raise MLAError("q rows must equal len(kv_len) * n_q")
+    if workspace is None:
+        need = int(lib.mla_decode_cudacore_workspace_bytes(B, n_q, H, num_splits))
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((T, H, D_H), dtype=torch.bfloat16, device=q.device)
+    _check(lib.mla_decode_cudacore(
+        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _ptr(cache, torch.bfloat16, None, "cache"), cache.shape[0],
+        _ptr(seq_start, torch.int64, (B,), "seq_start"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, float(scale), num_splits,
+        _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(out, torch.bfloat16, (T, H, D_H), "out"), _ptr(lse_out, torch.float32, (T, H), "lse_out"),
+        _ptr(dev_status, torch.int32, None, "dev_status"), _stream(stream)))
     return out
 
 

@@ -34,6 +34,39 @@ DecodeWs decode_ws_layout(int B, int n_q, int H, int S) {
 
 mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
+// ---- tensor-core path: segment partials [G][slots][128] x (float2 ml, 512 fp32 O)
+struct TcWs {
+    int G, slots;
+    size_t ml_part, o_part, total;
+};
+
+TcWs tc_ws_layout(int B, int n_q, int H) {
+    TcWs w;
+    w.G = (n_q * H + 127) / 128;
+    w.slots = B + decode_tc_max_clusters();
+    const size_t rows = static_cast<size_t>(w.G) * w.slots * 128;
+    w.ml_part = 0;
+    w.o_part = ((rows * sizeof(float2) + 1023) / 1024) * 1024;
+    w.total = w.o_part + rows * kDc * sizeof(float);
+    return w;
+}
+
+int tc_clusters_per_group(int G, int num_splits) {
+    const int total = decode_tc_clusters();
+    if (total <= 0) return 0;
+    int pg = total / G;
+    if (pg < 1) pg = 1;
+    if (num_splits > 0 && num_splits < pg) pg = num_splits;
+    return pg;
+}
+
+mla_status check_decode_shape(int B, int64_t cap_tokens, int n_q, int H, int num_splits) {
+    if (B < 0 || cap_tokens < 0 || cap_tokens >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+    if (H < 1 || H > kMaxHeads || n_q < 1 || n_q > kMaxNq || num_splits < 0 || num_splits > 256)
+        return MLA_ERR_UNSUPPORTED_SHAPE;
+    return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -103,44 +136,47 @@ mla_status mla_append_cache(void* cache, int64_t cap_tokens, const int64_t* seq_
 
 size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits) {
     if (B < 0 || n_q < 1 || H < 1 || num_splits < 0) return 0;
-    const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
-    return decode_ws_layout(B, n_q, H, S).total;
+    return tc_ws_layout(B, n_q, H).total;
 }
 
 mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_tokens, const int64_t* seq_start,
                              const int32_t* kv_len, int B, int n_q, int H, float scale, int num_splits,
                              void* workspace, size_t ws_bytes, int32_t* dev_status, mla_stream stream) {
-    if (B < 0 || cap_tokens < 0 || !(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
-    if (H < 1 || H > kMaxHeads || n_q < 1 || n_q > kMaxNq || num_splits < 0 || num_splits > 256)
-        return MLA_ERR_UNSUPPORTED_SHAPE;
+    mla_status st = check_decode_shape(B, cap_tokens, n_q, H, num_splits);
+    if (st != MLA_OK) return st;
+    if (!(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
     if (B == 0) return MLA_OK;
     if (!q || !cache || !seq_start || !kv_len || !workspace) return MLA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(cache) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
-    const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
-    const DecodeWs lay = decode_ws_layout(B, n_q, H, S);
+    const TcWs lay = tc_ws_layout(B, n_q, H);
     if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
-    float* o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.o_part);
-    float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.lse_part);
-    return cuda_status(launch_decode_simt(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(cache),
-                                          cap_tokens, seq_start, kv_len, B, n_q, H, scale, S, o_part, lse_part,
-                                          dev_status, static_cast<cudaStream_t>(stream)));
+    const int pg = tc_clusters_per_group(lay.G, num_splits);
+    if (pg <= 0) return MLA_ERR_CUDA;
+    char* ws = static_cast<char*>(workspace);
+    return cuda_status(launch_decode_tc(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(cache),
+                                        cap_tokens, seq_start, kv_len, B, n_q, H, scale, pg,
+                                        reinterpret_cast<float*>(ws + lay.o_part),
+                                        reinterpret_cast<float2*>(ws + lay.ml_part), lay.slots, dev_status,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
-mla_status mla_decode_finish(const void* W_UV, int B, int n_q, int H, int num_splits, void* workspace,
-                             size_t ws_bytes, void* out, float* lse_out, mla_stream stream) {
-    if (B < 0) return MLA_ERR_INVALID_ARG;
-    if (H < 1 || H > kMaxHeads || n_q < 1 || n_q > kMaxNq || num_splits < 0 || num_splits > 256)
-        return MLA_ERR_UNSUPPORTED_SHAPE;
+mla_status mla_decode_finish(const int64_t* seq_start, const int32_t* kv_len, int64_t cap_tokens, const void* W_UV,
+                             int B, int n_q, int H, int num_splits, void* workspace, size_t ws_bytes, void* out,
+                             float* lse_out, mla_stream stream) {
+    mla_status st = check_decode_shape(B, cap_tokens, n_q, H, num_splits);
+    if (st != MLA_OK) return st;
     if (B == 0) return MLA_OK;
-    if (!W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!seq_start || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
     if (!aligned16(W_UV) || !aligned16(out) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
-    const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
-    const DecodeWs lay = decode_ws_layout(B, n_q, H, S);
+    const TcWs lay = tc_ws_layout(B, n_q, H);
     if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
-    const float* o_part = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + lay.o_part);
-    const float* lse_part = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + lay.lse_part);
-    return cuda_status(launch_combine(o_part, lse_part, B * n_q, H, S, static_cast<const uint16_t*>(W_UV), out,
-                                      lse_out, static_cast<cudaStream_t>(stream)));
+    const int pg = tc_clusters_per_group(lay.G, num_splits);
+    if (pg <= 0) return MLA_ERR_CUDA;
+    const char* ws = static_cast<const char*>(workspace);
+    return cuda_status(launch_combine_tc(reinterpret_cast<const float*>(ws + lay.o_part),
+                                         reinterpret_cast<const float2*>(ws + lay.ml_part), kv_len, seq_start,
+                                         cap_tokens, B, n_q, H, pg, lay.slots, static_cast<const uint16_t*>(W_UV),
+                                         static_cast<uint16_t*>(out), lse_out, static_cast<cudaStream_t>(stream)));
 }
 
 mla_status mla_decode(const void* q, const void* cache, int64_t cap_tokens, const int64_t* seq_start,
@@ -152,7 +188,39 @@ mla_status mla_decode(const void* q, const void* cache, int64_t cap_tokens, cons
     mla_status st = mla_decode_attend(q, cache, cap_tokens, seq_start, kv_len, B, n_q, H, scale, num_splits,
                                       workspace, ws_bytes, dev_status, stream);
     if (st != MLA_OK || B == 0) return st;
-    return mla_decode_finish(W_UV, B, n_q, H, num_splits, workspace, ws_bytes, out, lse_out, stream);
+    return mla_decode_finish(seq_start, kv_len, cap_tokens, W_UV, B, n_q, H, num_splits, workspace, ws_bytes, out,
+                             lse_out, stream);
+}
+
+size_t mla_decode_cudacore_workspace_bytes(int B, int n_q, int H, int num_splits) {
+    if (B < 0 || n_q < 1 || H < 1 || num_splits < 0) return 0;
+    const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
+    return decode_ws_layout(B, n_q, H, S).total;
+}
+
+mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_tokens, const int64_t* seq_start,
+                               const int32_t* kv_len, const void* W_UV, int B, int n_q, int H, float scale,
+                               int num_splits, void* workspace, size_t ws_bytes, void* out, float* lse_out,
+                               int32_t* dev_status, mla_stream stream) {
+    mla_status st = check_decode_shape(B, cap_tokens, n_q, H, num_splits);
+    if (st != MLA_OK) return st;
+    if (!(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
+    if (B == 0) return MLA_OK;
+    if (!q || !cache || !seq_start || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(cache) || !aligned16(W_UV) || !aligned16(out) || !aligned16(workspace))
+        return MLA_ERR_INVALID_ARG;
+    const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
+    const DecodeWs lay = decode_ws_layout(B, n_q, H, S);
+    if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
+    float* o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.o_part);
+    float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.lse_part);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_decode_simt(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(cache),
+                                       cap_tokens, seq_start, kv_len, B, n_q, H, scale, S, o_part, lse_part,
+                                       dev_status, cs);
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    return cuda_status(launch_combine(o_part, lse_part, B * n_q, H, S, static_cast<const uint16_t*>(W_UV), out,
+                                      lse_out, cs));
 }
 
 mla_status mla_splitkv_combine(const float* o_part, const float* lse_part, int T, int H, int num_splits,

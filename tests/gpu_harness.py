@@ -51,10 +51,11 @@ class Problem:
     def absorb(self) -> torch.Tensor:
         return mla.absorb_q(self.q_nope, self.q_rope, self.q_pos, self.W_UK, self.rope_tab, dev_status=self.status)
 
-    def decode(self, q, num_splits=0, lse=True):
+    def decode(self, q, num_splits=0, lse=True, path="tc"):
         lse_out = torch.empty((self.T, self.cfg.H), dtype=torch.float32, device=q.device) if lse else None
-        out = mla.decode(q, self.cache, self.seq_start, self.kv_len, self.W_UV, self.cfg.n_q, self.cfg.scale,
-                         num_splits=num_splits, lse_out=lse_out, dev_status=self.status)
+        fn = mla.decode if path == "tc" else mla.decode_cudacore
+        out = fn(q, self.cache, self.seq_start, self.kv_len, self.W_UV, self.cfg.n_q, self.cfg.scale,
+                 num_splits=num_splits, lse_out=lse_out, dev_status=self.status)
         return out, lse_out
 
     def oracle(self, b: int, heads=None):
@@ -68,24 +69,26 @@ class Problem:
 
 
 def build_problem(cfg: mi.MLAConfig, lengths=None, slack_rows: int = 64, dev="cuda",
-                  chunk_rows: int = 1 << 16) -> Problem:
+                  chunk_rows: int = 1 << 16, gap_rows: int = 0) -> Problem:
     """Fill a packed cache with every sequence's tokens via mla_append_cache.
 
-    Sequences sit back to back from row 0; ``slack_rows`` extra rows at the end
-    hold NaN so that a kernel reading past a sequence would be noticed.
+    Sequences sit back to back from row 0 (or ``gap_rows`` apart); the gaps and
+    ``slack_rows`` extra rows at the end hold NaN so that a kernel reading past
+    a sequence would be noticed.
     """
     lengths = mi.kv_lengths(cfg) if lengths is None else np.asarray(lengths, dtype=np.int64)
-    starts = mi.seq_starts(lengths)
+    pool_starts = mi.seq_starts(lengths)            # rows in the generator's packed pool
+    starts = pool_starts + gap_rows * np.arange(cfg.B, dtype=np.int64)
     N = int(lengths.sum())
-    cache = torch.full((N + slack_rows, mi.D_ROW), 0, dtype=torch.int16, device=dev)
-    cache[N:] = NAN_BF16
+    cap = N + gap_rows * cfg.B + slack_rows
+    cache = torch.full((cap, mi.D_ROW), NAN_BF16, dtype=torch.int16, device=dev)
     cache = cache.view(torch.bfloat16)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     rope_tab = mla.rope_table(int(lengths.max()), cfg.rope_base, dev)
     seq_start = torch.from_numpy(starts).to(dev)
     # per-row (sequence, position) of the whole pool
     seq_of_row = np.repeat(np.arange(cfg.B, dtype=np.int32), lengths)
-    pos_of_row = (np.arange(N, dtype=np.int64) - np.repeat(starts, lengths)).astype(np.int32)
+    pos_of_row = (np.arange(N, dtype=np.int64) - np.repeat(pool_starts, lengths)).astype(np.int32)
     for r0 in range(0, N, chunk_rows):
         n = min(chunk_rows, N - r0)
         c, k = mi.token_rows(cfg, r0, n)

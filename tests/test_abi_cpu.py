@@ -80,8 +80,12 @@ def test_host_validation_rejects_bad_arguments(mla):
     assert L.mla_splitkv_combine(None, fake, 4, 16, 2, None, fake, None, None) == 1
 
 
-def test_workspace_grows_with_splits(mla):
+def test_workspace_sizes(mla):
+    # tensor-core path: one slot per (sequence + CTA pair) and row group, any split count
     a = mla.decode_workspace_bytes(32, 1, 128, 1)
-    b = mla.decode_workspace_bytes(32, 1, 128, 4)
-    assert b > a > 0
-    assert mla.decode_workspace_bytes(32, 1, 128, 0) > 0
+    assert a == mla.decode_workspace_bytes(32, 1, 128, 0) > 32 * 128 * 512 * 4
+    assert mla.decode_workspace_bytes(32, 2, 128, 0) > 1.9 * a
+    # CUDA-core path: one fp32 partial per split
+    c1 = mla.lib.mla_decode_cudacore_workspace_bytes(32, 1, 128, 1)
+    c4 = mla.lib.mla_decode_cudacore_workspace_bytes(32, 1, 128, 4)
+    assert c4 > 3.9 * c1 > 0

@@ -175,17 +175,44 @@ def test_decode_small_ragged_full(cuda_ok, H):
 
 @pytest.mark.parametrize("splits", [1, 2, 7, 32])
 def test_decode_split_invariance(cuda_ok, H, splits):
+    """Tensor-core path with at most `splits` CTA pairs per row group (so sequences
+    are cut into 1 .. many pieces) against the CUDA-core path and the oracle."""
     cfg = mi.MLAConfig("splits", B=3, H=32, n_q=2, L=None, L_max=3000, seed=55)
     prob = H.build_problem(cfg)
     q = prob.absorb()
-    ref_out, ref_lse = prob.decode(q, num_splits=1)
+    ref_out, ref_lse = prob.decode(q, num_splits=4, path="cudacore")
     out, lse = prob.decode(q, num_splits=splits)
     torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
     a, b = out.float().cpu().numpy(), ref_out.float().cpu().numpy()
-    # same math up to fp32 summation order, then one bf16 rounding
-    assert np.all(np.abs(a - b) <= 1e-4 + 2 ** -7 * np.abs(b))
-    assert np.abs(lse.cpu().numpy() - ref_lse.cpu().numpy()).max() < 1e-4
+    # same math up to summation order and the bf16 rounding of P
+    assert np.all(np.abs(a - b) <= 2e-3 + 2 ** -6 * np.abs(b))
+    assert np.abs(lse.cpu().numpy() - ref_lse.cpu().numpy()).max() < 1e-3
     _check_decode(prob, out, lse, [0, 2], label=f"splits={splits}")
+
+
+def test_decode_ignores_rows_outside_sequences(cuda_ok, H):
+    """NaN rows between and after sequences never leak into any result."""
+    cfg = mi.MLAConfig("gaps", B=5, H=128, n_q=2, L=None, L_max=400, seed=66)
+    prob = H.build_problem(cfg, gap_rows=37)
+    out, lse = prob.decode(prob.absorb())
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    assert torch.isfinite(out.float()).all()
+    _check_decode(prob, out, lse, range(cfg.B), heads=range(0, 128, 7), label="gaps")
+
+
+def test_decode_tensor_core_matches_cuda_core_path(cuda_ok, H):
+    cfg = mi.MLAConfig("paths", B=6, H=128, n_q=1, L=None, L_max=5000, seed=91)
+    prob = H.build_problem(cfg)
+    q = prob.absorb()
+    out_c, lse_c = prob.decode(q, path="cudacore")
+    out_t, lse_t = prob.decode(q)
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    a, b = out_t.float().cpu().numpy(), out_c.float().cpu().numpy()
+    assert np.all(np.abs(a - b) <= 2e-3 + 2 ** -6 * np.abs(b))
+    assert np.abs(lse_t.cpu().numpy() - lse_c.cpu().numpy()).max() < 1e-3
 
 
 @pytest.mark.parametrize("name,seqs,heads", [
