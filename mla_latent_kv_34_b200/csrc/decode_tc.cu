@@ -10,9 +10,10 @@
 //   CTA 0 ("S"): the 128 absorbed query rows live in TMEM (the A operand, 288
 //     columns); each 64-token tile of the cache is TMA-loaded (9 swizzled
 //     [64 x 64] chunks) and S = Q K^T is formed by 36 tcgen05.mma (M=128,
-//     N=64, K=16) into one of two TMEM score buffers.  Four warps (one thread
-//     per query row) run the online softmax in fp32 and write P (bf16) straight
-//     into CTA 1's shared memory over DSMEM.
+//     N=64, K=16) into one of two TMEM score buffers.  Eight warps (a query
+//     row's 64 scores split over two threads) run the online softmax in fp32,
+//     stage P (bf16) in shared memory, and one thread ships each P tile to
+//     CTA 1 with a single asynchronous bulk copy over DSMEM.
 //   CTA 1 ("O"): keeps the unnormalised latent output O[128 x 512] fp32 in its
 //     whole TMEM and accumulates O += P V with 8 tcgen05.mma (M=128, N=256,
 //     K=16) per tile; V is the first 512 columns of the same cache tile, read
@@ -45,45 +46,54 @@ using namespace sm100;
 
 namespace tc {
 
-constexpr int kTile = 64;           // tokens per tile
-constexpr int kRows = 128;          // query rows per CTA pair
+constexpr int kTile = 64;            // tokens per tile
+constexpr int kRows = 128;           // query rows per CTA pair
 constexpr int kChunk = 64 * 64 * 2;  // [64 tokens x 64 columns] bf16 = 8 KB
-constexpr int kKvChunks = 9;        // 576 / 64
-constexpr int kVChunks = 8;         // 512 / 64
-constexpr int kStagesS = 3;
-constexpr int kStagesO = 3;
-constexpr int kPBytes = kRows * kTile * 2;  // 16 KB bf16 P tile
-constexpr int kThreads = 192;
+constexpr int kKvChunks = 9;         // 576 / 64
+constexpr int kVChunks = 8;          // 512 / 64
+constexpr int kRing = 24;            // S CTA: ring of 8 KB cache chunks (2.67 tiles)
+constexpr int kStagesO = 3;          // O CTA: whole-tile V stages
+constexpr int kPrefetchTiles = 4;    // S CTA: tiles pulled into L2 ahead of the ring
+constexpr int kPBytes = kRows * kTile * 2;       // 16 KB bf16 P tile
+constexpr int kMsgBytes = kPBytes + kRows * 4 + 16;  // P | alpha[128] | flag (+pad): one bulk copy
+constexpr int kMsgStride = 17408;    // 1024-aligned message slots in the O CTA
+constexpr int kSoftWarps = 8;        // S CTA: two warps per TMEM lane quadrant
+constexpr int kSoftThreads = kSoftWarps * 32;
+constexpr int kWarpProducer = 8, kWarpMma = 9;
+constexpr int kThreads = 320;
 constexpr uint64_t kLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleLog2 = 8.0f;
 
 // TMEM columns (512 allocated in each CTA)
-constexpr uint32_t kColQ = 0;  // S CTA: Q rows, 288 columns of packed bf16 pairs
-constexpr uint32_t kColS0 = 384;  // two 64-column score buffers: 384 and 448
+constexpr uint32_t kColQ = 0;     // S CTA: Q rows, 288 columns of packed bf16 pairs
+constexpr uint32_t kColS0 = 384;  // S CTA: two 64-column score buffers (384, 448)
 __device__ __forceinline__ uint32_t col_s(uint32_t sb) { return kColS0 + 64u * sb; }
 
-// shared memory layout (identical offsets in both CTAs so that mapa works)
-constexpr int kOffKv = 0;                                    // S: 3 x 9 x 8 KB
-constexpr int kOffV = 0;                                     // O: 3 x 8 x 8 KB
-constexpr int kOffP = kStagesO * kVChunks * kChunk;          // O: 2 x 16 KB
-constexpr int kOffAlpha = kOffP + 2 * kPBytes;               // O: 2 x 128 fp32
-constexpr int kOffFlag = kOffAlpha + 2 * kRows * 4;          // O: 2 x u32
-constexpr int kOffBar = kOffFlag + 16;                       // 16 mbarriers
-constexpr int kOffTail = kOffBar + 16 * 8;                   // tmem base, abort, misc
-constexpr int kSmemBytes = kOffTail + 32;
-static_assert(kStagesS * kKvChunks * kChunk <= kOffBar, "S data overlaps barriers");
+// shared memory, S CTA
+constexpr int kSOffRing = 0;                                  // 24 x 8 KB
+constexpr int kSOffStage = kRing * kChunk;                    // 2 x kMsgBytes (local P messages)
+constexpr int kSOffXchg = kSOffStage + 2 * kMsgBytes;         // [2][128] fp32 half-row maxima / sums
+constexpr int kSOffBar = kSOffXchg + 2 * kRows * 4;
+// barrier slots, S CTA: a tile's chunks arrive together (one or two TMA boxes) on
+// kSBarTFull[tile % 3]; ring slots are released one chunk at a time.
+constexpr int kTilesInRing = 3;  // at most 3 tiles own ring slots at any time (24 / 9 rounded up)
+constexpr int kSBarTFull = 0, kSBarEmpty = kTilesInRing, kSBarSFull = kSBarEmpty + kRing,
+              kSBarSEmpty = kSBarSFull + 2, kSBarPEmpty = kSBarSEmpty + 2, kSBarQReady = kSBarPEmpty + 2,
+              kSBarFin = kSBarQReady + 1, kSNumBars = kSBarFin + 1;
+constexpr int kSOffTail = kSOffBar + kSNumBars * 8;
+// shared memory, O CTA
+constexpr int kOOffV = 0;                                     // 3 x 8 x 8 KB
+constexpr int kOOffMsg = kStagesO * kVChunks * kChunk;        // 2 message slots
+constexpr int kOOffBar = kOOffMsg + 2 * kMsgStride;
+constexpr int kOBarVFull = 0, kOBarVEmpty = kStagesO, kOBarPFull = 2 * kStagesO, kOBarOFull = kOBarPFull + 2,
+              kOBarOFree = kOBarOFull + 1, kOBarRescReq = kOBarOFree + 1, kOBarRescDone = kOBarRescReq + 1,
+              kOBarODrain = kOBarRescDone + 1, kOBarFin = kOBarODrain + 1, kONumBars = kOBarFin + 1;
+constexpr int kOOffTail = kOOffBar + kONumBars * 8;
+constexpr int kTailBytes = 32;  // tmem base, abort flag, resc slot, tile total
+constexpr int kSmemBytes = (kSOffTail > kOOffTail ? kSOffTail : kOOffTail) + kTailBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-
-// barrier slots
-enum : int {
-    // S CTA
-    kBarKvFull = 0, kBarKvEmpty = 3, kBarSFull = 6, kBarSEmpty = 8, kBarPEmpty = 10, kBarQReady = 12,
-    // O CTA
-    kBarVFull = 0, kBarVEmpty = 3, kBarPFull = 6, kBarOFull = 8, kBarOFree = 9, kBarRescReq = 10,
-    kBarRescDone = 11, kBarODrain = 12,
-    // both
-    kBarFin = 13
-};
+static_assert(kSOffStage % 16 == 0 && kMsgBytes % 16 == 0, "bulk copy alignment");
+static_assert(kOOffMsg % 1024 == 0 && kMsgStride % 1024 == 0, "P tiles must be 1024-byte aligned");
 
 struct Params {
     const uint16_t* q;
@@ -153,18 +163,32 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t p
     if (dev_status) atomicOr(dev_status, MLA_DEVERR_TIMEOUT);
 }
 
+__device__ __forceinline__ float fmax32(const float (&v)[32]) {
+    float a = fmaxf(v[0], v[1]), b = fmaxf(v[2], v[3]), c = fmaxf(v[4], v[5]), d = fmaxf(v[6], v[7]);
+#pragma unroll
+    for (int k = 8; k < 32; k += 4) {
+        a = fmaxf(a, v[k]);
+        b = fmaxf(b, v[k + 1]);
+        c = fmaxf(c, v[k + 2]);
+        d = fmaxf(d, v[k + 3]);
+    }
+    return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
+decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant__ CUtensorMap kv6,
+                 const __grid_constant__ CUtensorMap kv3, const __grid_constant__ CUtensorMap v8, const Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();  // 0: S CTA, 1: O CTA
     const uint32_t peer = rank ^ 1u;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTail);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffTail + 4);
-    volatile int* resc_pb = reinterpret_cast<volatile int*>(smem + kOffTail + 8);
-    int* nt_total = reinterpret_cast<int*>(smem + kOffTail + 12);
+    const int tail = rank == 0 ? kSOffTail : kOOffTail;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (rank == 0 ? kSOffBar : kOOffBar));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + tail);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + tail + 4);
+    volatile int* resc_pb = reinterpret_cast<volatile int*>(smem + tail + 8);
+    int* nt_total = reinterpret_cast<int*>(smem + tail + 12);
     volatile int never = 0;  // abort flag for teardown waits (never raised)
 
     if ((sbase & 1023u) != 0) {  // identical in both CTAs: both leave here
@@ -173,29 +197,28 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
     }
     if (tid == 0) {
         if (rank == 0) {
-            for (int i = 0; i < kStagesS; ++i) {
-                mbar_init(&bars[kBarKvFull + i], 1);
-                mbar_init(&bars[kBarKvEmpty + i], 1);
-            }
+            for (int i = 0; i < kTilesInRing; ++i) mbar_init(&bars[kSBarTFull + i], 1);
+            for (int i = 0; i < kRing; ++i) mbar_init(&bars[kSBarEmpty + i], 1);
             for (int i = 0; i < 2; ++i) {
-                mbar_init(&bars[kBarSFull + i], 1);
-                mbar_init(&bars[kBarSEmpty + i], kRows);
-                mbar_init(&bars[kBarPEmpty + i], 1);
+                mbar_init(&bars[kSBarSFull + i], 1);
+                mbar_init(&bars[kSBarSEmpty + i], kSoftThreads);
+                mbar_init(&bars[kSBarPEmpty + i], 1);
             }
-            mbar_init(&bars[kBarQReady], kRows);
+            mbar_init(&bars[kSBarQReady], kSoftThreads);
+            mbar_init(&bars[kSBarFin], 1);
         } else {
             for (int i = 0; i < kStagesO; ++i) {
-                mbar_init(&bars[kBarVFull + i], 1);
-                mbar_init(&bars[kBarVEmpty + i], 1);
+                mbar_init(&bars[kOBarVFull + i], 1);
+                mbar_init(&bars[kOBarVEmpty + i], 1);
             }
-            for (int i = 0; i < 2; ++i) mbar_init(&bars[kBarPFull + i], kRows);
-            mbar_init(&bars[kBarOFull], 1);
-            mbar_init(&bars[kBarOFree], kRows);
-            mbar_init(&bars[kBarRescReq], 1);
-            mbar_init(&bars[kBarRescDone], kRows);
-            mbar_init(&bars[kBarODrain], 1);
+            for (int i = 0; i < 2; ++i) mbar_init(&bars[kOBarPFull + i], 1);
+            mbar_init(&bars[kOBarOFull], 1);
+            mbar_init(&bars[kOBarOFree], kRows);
+            mbar_init(&bars[kOBarRescReq], 1);
+            mbar_init(&bars[kOBarRescDone], kRows);
+            mbar_init(&bars[kOBarODrain], 1);
+            mbar_init(&bars[kOBarFin], 1);
         }
-        mbar_init(&bars[kBarFin], 1);
         *abort_flag = 0;
         *resc_pb = 0;
         fence_mbar_init();
@@ -215,7 +238,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         if (lane == 0) *nt_total = s;
     }
-    if (warp == 4) tmem_alloc(tmem_slot, 512);
+    if (warp == kWarpProducer) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -227,181 +250,250 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
     const bool active = g < p.G;
     const int lo = static_cast<int>((static_cast<int64_t>(pidx) * Nt) / p.P_g);
     const int hi = static_cast<int>((static_cast<int64_t>(pidx + 1) * Nt) / p.P_g);
-    const uint32_t peer_abort = mapa(sbase + kOffTail + 4, peer);
+    const uint32_t peer_abort = mapa(sbase + (rank == 0 ? kOOffTail : kSOffTail) + 4, peer);
     const int64_t out_row_base = (static_cast<int64_t>(g) * p.slots) * kRows;
 
     if (active && rank == 0) {
         // =============================================================== S CTA
-        if (warp == 4) {
-            // ---- TMA producer: one 64-token tile = 9 chunks of [64 tokens x 64 cols]
+        if (warp == kWarpProducer) {
+            // ---- TMA producer.  The cache is viewed as a 3-D tensor (column in chunk, token,
+            //      chunk) so that one box lands a whole 64-token tile chunk-major in the
+            //      24-slot ring (a tile that wraps the ring end takes two boxes: 6 + 3 or
+            //      3 + 6 chunks).  A second walker pulls tiles kPrefetchTiles ahead into L2.
             if (lane == 0) {
-                prefetch_tmap(&kv_map);
-                SegWalk w;
+                prefetch_tmap(&kv9);
+                prefetch_tmap(&kv6);
+                prefetch_tmap(&kv3);
+                SegWalk w, wp;
                 w.init(p, lo, hi, pidx);
-                Seg s;
-                uint32_t n = 0;
+                wp.init(p, lo, hi, pidx);
+                Seg s, sp;
+                bool have_p = wp.next(p, sp);
+                int tp = have_p ? sp.t0 : 0;
+                auto prefetch_one = [&]() {
+                    if (!have_p) return;
+                    tma_prefetch_3d(&kv9, 0, static_cast<int>(sp.row0 + static_cast<int64_t>(tp) * kTile), 0);
+                    if (++tp >= sp.t1) {
+                        have_p = wp.next(p, sp);
+                        tp = have_p ? sp.t0 : 0;
+                    }
+                };
+                for (int i = 0; i < kPrefetchTiles; ++i) prefetch_one();
+                uint32_t n = 0;  // tiles issued
                 bool ok = true;
                 while (ok && w.next(p, s)) {
-                    for (int t = s.t0; t < s.t1; ++t, ++n) {
-                        const uint32_t st = n % kStagesS, u = n / kStagesS;
-                        if (!mbar_wait(&bars[kBarKvEmpty + st], (u & 1u) ^ 1u, abort_flag, kLimitNs)) {
-                            ok = false;
-                            break;
+                    for (int t = s.t0; ok && t < s.t1; ++t, ++n) {
+                        prefetch_one();
+                        const uint32_t gc = n * kKvChunks, s0 = gc % kRing;
+                        for (int c = 0; ok && c < kKvChunks; ++c) {
+                            const uint32_t g2 = gc + c;
+                            ok = mbar_wait(&bars[kSBarEmpty + g2 % kRing], ((g2 / kRing) & 1u) ^ 1u, abort_flag, kLimitNs);
                         }
-                        mbar_arrive_expect_tx(&bars[kBarKvFull + st], kKvChunks * kChunk);
+                        if (!ok) break;
+                        uint64_t* tb = &bars[kSBarTFull + n % kTilesInRing];
+                        mbar_arrive_expect_tx(tb, kKvChunks * kChunk);
                         const int y = static_cast<int>(s.row0 + static_cast<int64_t>(t) * kTile);
-#pragma unroll
-                        for (int c = 0; c < kKvChunks; ++c)
-                            tma_load_2d(sbase + kOffKv + (st * kKvChunks + c) * kChunk, &kv_map, 64 * c, y,
-                                        &bars[kBarKvFull + st]);
+                        const uint32_t dst = sbase + kSOffRing + s0 * kChunk;
+                        if (s0 + kKvChunks <= static_cast<uint32_t>(kRing)) {
+                            tma_load_3d(dst, &kv9, 0, y, 0, tb);
+                        } else {
+                            const uint32_t first = kRing - s0;  // 6 or 3 chunks up to the ring end
+                            tma_load_3d(dst, first == 6 ? &kv6 : &kv3, 0, y, 0, tb);
+                            tma_load_3d(sbase + kSOffRing, first == 6 ? &kv3 : &kv6, 0, y, static_cast<int>(first), tb);
+                        }
                     }
                 }
                 if (!ok) raise_abort(abort_flag, peer_abort, p.dev_status);
                 // let every issued copy land before the CTA can exit
-                for (uint32_t i = (n > kStagesS ? n - kStagesS : 0); i < n; ++i)
-                    mbar_wait(&bars[kBarKvFull + i % kStagesS], (i / kStagesS) & 1u, &never, kLimitNs);
+                for (uint32_t i = (n > kTilesInRing ? n - kTilesInRing : 0); i < n; ++i)
+                    mbar_wait(&bars[kSBarTFull + i % kTilesInRing], (i / kTilesInRing) & 1u, &never, kLimitNs);
             }
-        } else if (warp == 5) {
-            // ---- MMA issuer: S[sb] = Q K^T (A from TMEM, B = cache tile, K-major SW128)
-            constexpr uint32_t idesc = idesc_bf16_f32(kRows, kTile, false, false);
-            SegWalk w;
-            w.init(p, lo, hi, pidx);
-            Seg s;
-            uint32_t n = 0, kseg = 0;
-            bool ok = true;
-            while (ok && w.next(p, s)) {
-                ok = mbar_wait(&bars[kBarQReady], kseg & 1u, abort_flag, kLimitNs);
-                ++kseg;
-                for (int t = s.t0; ok && t < s.t1; ++t, ++n) {
-                    const uint32_t st = n % kStagesS, u = n / kStagesS;
-                    const uint32_t sb = n & 1u, us = n >> 1;
-                    ok = mbar_wait(&bars[kBarKvFull + st], u & 1u, abort_flag, kLimitNs) &&
-                         mbar_wait(&bars[kBarSEmpty + sb], (us & 1u) ^ 1u, abort_flag, kLimitNs);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (lane == 0) {
+        } else if (warp == kWarpMma) {
+            // ---- MMA issuer (one thread): S[sb] = Q K^T, A from TMEM, B = cache chunks
+            //      (K-major SW128).  Once a tile has landed its 36 MMAs go out back to back;
+            //      each chunk's ring slot is released (commit) as soon as its 4 MMAs finish.
+            if (lane == 0) {
+                constexpr uint32_t idesc = idesc_bf16_f32(kRows, kTile, false, false);
+                const uint64_t ring_desc = sdesc_sw128(sbase + kSOffRing, 16, 1024);
+                SegWalk w;
+                w.init(p, lo, hi, pidx);
+                Seg s;
+                uint32_t n = 0, kseg = 0, gc = 0;
+                bool ok = true;
+                while (ok && w.next(p, s)) {
+                    ok = mbar_wait(&bars[kSBarQReady], kseg & 1u, abort_flag, kLimitNs);
+                    ++kseg;
+                    for (int t = s.t0; ok && t < s.t1; ++t, ++n, gc += kKvChunks) {
+                        const uint32_t sb = n & 1u, us = n >> 1;
+                        ok = mbar_wait(&bars[kSBarSEmpty + sb], (us & 1u) ^ 1u, abort_flag, kLimitNs) &&
+                             mbar_wait(&bars[kSBarTFull + n % kTilesInRing], (n / kTilesInRing) & 1u, abort_flag,
+                                       kLimitNs);
+                        if (!ok) break;
+                        tc_fence_after();
                         const uint32_t d = tmem + col_s(sb);
-                        const uint32_t kv = sbase + kOffKv + st * kKvChunks * kChunk;
 #pragma unroll
-                        for (int k = 0; k < kRow / 16; ++k) {
-                            const uint64_t bd = sdesc_sw128(kv + (k >> 2) * kChunk + (k & 3) * 32, 16, 1024);
-                            mma_ts(d, tmem + kColQ + 8 * k, bd, idesc, k > 0 ? 1u : 0u);
+                        for (int c = 0; c < kKvChunks; ++c) {
+                            const uint32_t slot = (gc + c) % kRing;
+                            const uint64_t cd = ring_desc + (static_cast<uint64_t>(slot * kChunk) >> 4);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                mma_ts(d, tmem + kColQ + 8 * (4 * c + k), cd + 2 * k, idesc, (c | k) ? 1u : 0u);
+                            mma_commit(smem_u32(&bars[kSBarEmpty + slot]));  // slot free once these 4 finish
                         }
-                        mma_commit(smem_u32(&bars[kBarSFull + sb]));
-                        mma_commit(smem_u32(&bars[kBarKvEmpty + st]));
+                        mma_commit(smem_u32(&bars[kSBarSFull + sb]));
                     }
-                    __syncwarp();
                 }
+                if (!ok) raise_abort(abort_flag, peer_abort, p.dev_status);
+                mma_commit(smem_u32(&bars[kSBarFin]));
+                mbar_wait(&bars[kSBarFin], 0, &never, kLimitNs);
             }
-            if (!ok && lane == 0) raise_abort(abort_flag, peer_abort, p.dev_status);
-            if (lane == 0) mma_commit(smem_u32(&bars[kBarFin]));
-            mbar_wait(&bars[kBarFin], 0, &never, kLimitNs);
+            __syncwarp();
         } else {
-            // ---- softmax: warps 0..3, one thread per query row
-            const int r = tid;
-            const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-            const uint32_t peer_p = mapa(sbase + kOffP, peer);
-            const uint32_t peer_alpha = mapa(sbase + kOffAlpha, peer);
-            const uint32_t peer_flag = mapa(sbase + kOffFlag, peer);
-            const uint32_t peer_pfull = mapa(smem_u32(&bars[kBarPFull]), peer);
+            // ---- softmax: 8 warps; warp (q, hf) owns TMEM lanes 32q.. (query rows) and
+            //      score columns 32hf .. 32hf + 31 of each 64-token tile
+            const int qd = warp & 3, hf = warp >> 2;
+            const int r = 32 * qd + lane;
+            const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * qd) << 16);
+            float* xchg = reinterpret_cast<float*>(smem + kSOffXchg);  // [2][128]
+            const uint32_t peer_msg = mapa(sbase + kOOffMsg, peer);
+            const uint32_t peer_pfull = mapa(sbase + kOOffBar + kOBarPFull * 8, peer);
             const int rr = g * kRows + r;
             const bool row_ok = rr < p.R;
             const int j = row_ok ? rr / p.H : 0;
-            SegWalk w;
+            SegWalk w, wn;
             w.init(p, lo, hi, pidx);
-            Seg s;
+            Seg s, sn;
             uint32_t n = 0;
             bool failed = false;
-            while (!failed && w.next(p, s)) {
-                // this segment's absorbed query row -> TMEM columns 0..287
-                __syncwarp();
+            bool have = w.next(p, s);
+            while (!failed && have) {
+                wn = w;
+                const bool have_next = wn.next(p, sn);
+                // this segment's absorbed query row -> TMEM columns 0..287 (warp hf=0: chunks 0..4,
+                // hf=1: chunks 5..8); the next segment's rows are prefetched into L2
                 const uint16_t* qrow = p.q + (static_cast<int64_t>(s.b) * p.R + (row_ok ? rr : 0)) * kRow;
-#pragma unroll 1
-                for (int c = 0; c < kKvChunks; ++c) {
-                    uint32_t v[32];
-                    const uint4* src = reinterpret_cast<const uint4*>(qrow + 64 * c);
+                if (have_next && row_ok) {
+                    const char* nq = reinterpret_cast<const char*>(p.q + (static_cast<int64_t>(sn.b) * p.R + rr) * kRow);
+                    for (int c = hf; c < 9; c += 2) prefetch_l2(nq + 128 * c);
+                }
+                __syncwarp();
+                {
+                    const int c0 = hf ? 5 : 0, c1 = hf ? 9 : 5;
+                    for (int c = c0; c < c1; c += 2) {
+                        uint32_t v0[32], v1[32];
+                        const uint4* src = reinterpret_cast<const uint4*>(qrow + 64 * c);
+                        const bool two = (c + 1) < c1;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint4 x = row_ok ? src[k] : make_uint4(0, 0, 0, 0);
-                        v[4 * k] = x.x;
-                        v[4 * k + 1] = x.y;
-                        v[4 * k + 2] = x.z;
-                        v[4 * k + 3] = x.w;
+                        for (int k = 0; k < 8; ++k) {
+                            const uint4 x = row_ok ? src[k] : make_uint4(0, 0, 0, 0);
+                            const uint4 y = (row_ok && two) ? src[k + 8] : make_uint4(0, 0, 0, 0);
+                            v0[4 * k] = x.x; v0[4 * k + 1] = x.y; v0[4 * k + 2] = x.z; v0[4 * k + 3] = x.w;
+                            v1[4 * k] = y.x; v1[4 * k + 1] = y.y; v1[4 * k + 2] = y.z; v1[4 * k + 3] = y.w;
+                        }
+                        tmem_st32(t_lane + kColQ + 32 * c, v0);
+                        if (two) tmem_st32(t_lane + kColQ + 32 * (c + 1), v1);
                     }
-                    tmem_st32(t_lane + kColQ + 32 * c, v);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars[kBarQReady]);
+                mbar_arrive(&bars[kSBarQReady]);
                 const int lim = row_ok ? (s.L - p.n_q + j + 1) : 0;  // keys 0 .. lim-1 are visible
                 float m = -CUDART_INF_F, l = 0.f;
                 for (int t = s.t0; t < s.t1; ++t, ++n) {
                     const uint32_t sb = n & 1u, us = n >> 1;
-                    bool ok = mbar_wait(&bars[kBarSFull + sb], us & 1u, abort_flag, kLimitNs);
+                    bool ok = mbar_wait(&bars[kSBarSFull + sb], us & 1u, abort_flag, kLimitNs);
                     __syncwarp();
                     tc_fence_after();
-                    uint32_t a0[32], a1[32];
-                    tmem_ld32(t_lane + col_s(sb), a0);
-                    tmem_ld32(t_lane + col_s(sb) + 32, a1);
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(&bars[kBarSEmpty + sb]);
-                    const int nvalid = max(0, min(kTile, lim - t * kTile));
-                    float x[kTile];
+                    float sv[32];
+                    {
+                        uint32_t a[32];
+                        tmem_ld32(t_lane + col_s(sb) + 32 * hf, a);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        x[k] = k < nvalid ? __uint_as_float(a0[k]) * p.scale_log2 : -CUDART_INF_F;
-                        x[k + 32] = (k + 32) < nvalid ? __uint_as_float(a1[k]) * p.scale_log2 : -CUDART_INF_F;
+                        for (int k = 0; k < 32; ++k) sv[k] = __uint_as_float(a[k]);
                     }
-                    float tmax = x[0];
+                    tc_fence_before();
+                    mbar_arrive(&bars[kSBarSEmpty + sb]);
+                    const int nvalid = lim - t * kTile - 32 * hf;  // columns < nvalid are visible
+                    if (nvalid < 32) {
 #pragma unroll
-                    for (int k = 1; k < kTile; ++k) tmax = fmaxf(tmax, x[k]);
+                        for (int k = 0; k < 32; ++k) sv[k] = k < nvalid ? sv[k] : -CUDART_INF_F;
+                    }
+                    // row max over both halves (raw scores; the scale is positive)
+                    xchg[hf * kRows + r] = fmax32(sv);
+                    bar_sync(1 + qd, 64);
+                    const float tmax = fmaxf(xchg[r], xchg[kRows + r]) * p.scale_log2;
                     const bool resc = tmax > m + kRescaleLog2;
                     float alpha = 1.f;
                     if (resc) {
-                        alpha = (m == -CUDART_INF_F) ? 0.f : exp2f(m - tmax);
+                        alpha = (m == -CUDART_INF_F) ? 0.f : ex2_approx(m - tmax);
                         l *= alpha;
                         m = tmax;
                     }
-                    const float mref = (m == -CUDART_INF_F) ? 0.f : m;
-                    uint32_t pk[32];
+                    const float mneg = (m == -CUDART_INF_F) ? 0.f : -m;
+                    uint32_t pk[16];
                     float lsum = 0.f;
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const float p0 = exp2f(x[2 * k] - mref), p1 = exp2f(x[2 * k + 1] - mref);
+                    for (int k = 0; k < 16; ++k) {
+                        const float p0 = ex2_approx(fmaf(sv[2 * k], p.scale_log2, mneg));
+                        const float p1 = ex2_approx(fmaf(sv[2 * k + 1], p.scale_log2, mneg));
                         lsum += p0 + p1;
-                        pk[k] = pack_bf16x2(p0, p1);
+                        pk[k] = cvt_bf16x2(p0, p1);
                     }
                     l += lsum;
-                    ok = ok && mbar_wait<true>(&bars[kBarPEmpty + sb], (us & 1u) ^ 1u, abort_flag, kLimitNs);
-                    if (bar_red_or(1, kRows, !ok || *abort_flag != 0)) {
+                    // staging slot sb is free once the bulk copy of two tiles ago has read it
+                    if (tid == 0 && n >= 2) bulk_wait_group_read<1>();
+                    const bool flag = bar_red_or(5, kSoftThreads, resc && t != s.t0);
+                    uint8_t* msg = smem + kSOffStage + sb * kMsgBytes;
+                    {
+                        // P row r, columns 32hf.. : 16-byte units 4hf..4hf+3, 128-byte swizzle
+                        uint8_t* prow = msg + r * 128;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int uu = 4 * hf + u;
+                            *reinterpret_cast<uint4*>(prow + ((uu ^ (r & 7)) << 4)) =
+                                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                        }
+                        if (hf == 0) reinterpret_cast<float*>(msg + kPBytes)[r] = alpha;
+                        if (tid == 0) *reinterpret_cast<uint32_t*>(msg + kPBytes + kRows * 4) = flag ? 1u : 0u;
+                    }
+                    fence_proxy_async_cta();
+                    if (bar_red_or(6, kSoftThreads, !ok || *abort_flag != 0)) {
                         failed = true;
                         break;
                     }
-                    const bool flag = bar_red_or(2, kRows, resc && t != s.t0);
-                    // P row r -> peer's P buffer (K-major, 128-byte swizzle: unit u at u ^ (r & 7))
-                    const uint32_t prow = peer_p + sb * kPBytes + r * 128;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        st_cluster_v4(prow + ((u ^ (r & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
-                                      pk[4 * u + 3]);
-                    st_cluster_f32(peer_alpha + sb * kRows * 4 + 4 * r, alpha);
-                    if (r == 0) st_cluster_u32(peer_flag + 4 * sb, flag ? 1u : 0u);
-                    fence_proxy_async_cluster();
-                    mbar_arrive_remote(peer_pfull + 8 * sb);
+                    if (tid == 0) {
+                        // ship the message once the O CTA has finished with this slot
+                        if (mbar_wait<true>(&bars[kSBarPEmpty + sb], (us & 1u) ^ 1u, abort_flag, kLimitNs)) {
+                            mbar_arrive_expect_tx_remote(peer_pfull + 8 * sb, kMsgBytes);
+                            bulk_copy_to_peer(peer_msg + sb * kMsgStride, sbase + kSOffStage + sb * kMsgBytes, kMsgBytes,
+                                              peer_pfull + 8 * sb);
+                            bulk_commit_group();
+                        } else {
+                            raise_abort(abort_flag, peer_abort, p.dev_status);
+                        }
+                    }
                 }
                 if (failed) break;
-                if (row_ok) p.ml_part[out_row_base + static_cast<int64_t>(s.slot) * kRows + r] = make_float2(m, l);
+                // segment result: (m, l) with l summed over both column halves
+                if (hf == 1) xchg[kRows + r] = l;
+                bar_sync(1 + qd, 64);
+                if (hf == 0 && row_ok)
+                    p.ml_part[out_row_base + static_cast<int64_t>(s.slot) * kRows + r] = make_float2(m, l + xchg[kRows + r]);
+                bar_sync(1 + qd, 64);
+                w = wn;
+                s = sn;
+                have = have_next;
             }
-            if (failed && r == 0) raise_abort(abort_flag, peer_abort, p.dev_status);
+            if (failed && tid == 0) raise_abort(abort_flag, peer_abort, p.dev_status);
+            if (tid == 0) bulk_wait_group_read<0>();
         }
     } else if (active && rank == 1) {
         // =============================================================== O CTA
-        if (warp == 4) {
+        if (warp == kWarpProducer) {
             // ---- TMA producer: the 8 latent chunks of each tile (V)
             if (lane == 0) {
-                prefetch_tmap(&kv_map);
+                prefetch_tmap(&v8);
                 SegWalk w;
                 w.init(p, lo, hi, pidx);
                 Seg s;
@@ -410,27 +502,25 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
                 while (ok && w.next(p, s)) {
                     for (int t = s.t0; t < s.t1; ++t, ++n) {
                         const uint32_t st = n % kStagesO, u = n / kStagesO;
-                        if (!mbar_wait(&bars[kBarVEmpty + st], (u & 1u) ^ 1u, abort_flag, kLimitNs)) {
+                        if (!mbar_wait(&bars[kOBarVEmpty + st], (u & 1u) ^ 1u, abort_flag, kLimitNs)) {
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&bars[kBarVFull + st], kVChunks * kChunk);
+                        mbar_arrive_expect_tx(&bars[kOBarVFull + st], kVChunks * kChunk);
                         const int y = static_cast<int>(s.row0 + static_cast<int64_t>(t) * kTile);
-#pragma unroll
-                        for (int c = 0; c < kVChunks; ++c)
-                            tma_load_2d(sbase + kOffV + (st * kVChunks + c) * kChunk, &kv_map, 64 * c, y,
-                                        &bars[kBarVFull + st]);
+                        tma_load_3d(sbase + kOOffV + st * kVChunks * kChunk, &v8, 0, y, 0, &bars[kOBarVFull + st]);
                     }
                 }
                 if (!ok) raise_abort(abort_flag, peer_abort, p.dev_status);
                 for (uint32_t i = (n > kStagesO ? n - kStagesO : 0); i < n; ++i)
-                    mbar_wait(&bars[kBarVFull + i % kStagesO], (i / kStagesO) & 1u, &never, kLimitNs);
+                    mbar_wait(&bars[kOBarVFull + i % kStagesO], (i / kStagesO) & 1u, &never, kLimitNs);
             }
-        } else if (warp == 5) {
-            // ---- MMA issuer: O += P V (A = P, K-major SW128; B = V, MN-major SW128)
+        } else if (warp == kWarpMma) {
+            // ---- MMA issuer (one thread): O += P V (A = P, K-major SW128; B = V, MN-major SW128)
             constexpr uint32_t idesc = idesc_bf16_f32(kRows, 256, false, true);
-            const uint32_t peer_pempty = mapa(smem_u32(&bars[kBarPEmpty]), peer);
-            volatile uint32_t* flags = reinterpret_cast<volatile uint32_t*>(smem + kOffFlag);
+            const uint32_t peer_pempty = mapa(sbase + kSOffBar + kSBarPEmpty * 8, peer);
+            const uint64_t p_desc = sdesc_sw128(sbase + kOOffMsg, 16, 1024);
+            const uint64_t v_desc = sdesc_sw128(sbase + kOOffV, kChunk, 1024);
             SegWalk w;
             w.init(p, lo, hi, pidx);
             Seg s;
@@ -441,28 +531,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
                     const uint32_t st = n % kStagesO, u = n / kStagesO;
                     const uint32_t pb = n & 1u, up = n >> 1;
                     const bool first = (t == s.t0);
-                    ok = mbar_wait(&bars[kBarVFull + st], u & 1u, abort_flag, kLimitNs) &&
-                         mbar_wait<true>(&bars[kBarPFull + pb], up & 1u, abort_flag, kLimitNs);
-                    if (ok && first) ok = mbar_wait(&bars[kBarOFree], (kseg & 1u) ^ 1u, abort_flag, kLimitNs);
-                    ok = __all_sync(0xffffffffu, ok);
+                    if (lane == 0) {
+                        ok = mbar_wait(&bars[kOBarVFull + st], u & 1u, abort_flag, kLimitNs) &&
+                             mbar_wait<true>(&bars[kOBarPFull + pb], up & 1u, abort_flag, kLimitNs);
+                        if (ok && first) ok = mbar_wait(&bars[kOBarOFree], (kseg & 1u) ^ 1u, abort_flag, kLimitNs);
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
-                    if (!first && flags[pb] != 0u) {
+                    const uint8_t* msg = smem + kOOffMsg + pb * kMsgStride;
+                    if (!first && *reinterpret_cast<const volatile uint32_t*>(msg + kPBytes + kRows * 4) != 0u) {
                         // stale max moved: have the epilogue rescale O once all earlier MMAs are done
                         if (lane == 0) {
                             *resc_pb = static_cast<int>(pb);
-                            mma_commit(smem_u32(&bars[kBarODrain]));
-                            mbar_arrive(&bars[kBarRescReq]);
+                            mma_commit(smem_u32(&bars[kOBarODrain]));
+                            mbar_arrive(&bars[kOBarRescReq]);
+                            ok = mbar_wait(&bars[kOBarRescDone], nresc & 1u, abort_flag, kLimitNs);
                         }
-                        __syncwarp();
-                        ok = __all_sync(0xffffffffu,
-                                        mbar_wait(&bars[kBarRescDone], nresc & 1u, abort_flag, kLimitNs));
                         ++nresc;
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
                         if (!ok) break;
                     }
                     const int nvalid = min(kTile, s.L - t * kTile);
                     if (nvalid < kTile) {
                         // rows past the sequence end: P is 0 there, make V 0 too (no 0 * NaN)
-                        uint8_t* vst = smem + kOffV + st * kVChunks * kChunk;
+                        uint8_t* vst = smem + kOOffV + st * kVChunks * kChunk;
                         const int nz = (kTile - nvalid) * 8;  // 16-byte units per chunk
                         for (int i = lane; i < kVChunks * nz; i += 32) {
                             const int c = i / nz, k = i % nz;
@@ -471,37 +563,37 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
                         fence_proxy_async_cta();
                         __syncwarp();
                     }
-                    tc_fence_after();
                     if (lane == 0) {
-                        const uint32_t pa = sbase + kOffP + pb * kPBytes;
-                        const uint32_t vb = sbase + kOffV + st * kVChunks * kChunk;
+                        tc_fence_after();
+                        const uint64_t pd = p_desc + (static_cast<uint64_t>(pb * kMsgStride) >> 4);
+                        const uint64_t vd = v_desc + (static_cast<uint64_t>(st * kVChunks * kChunk) >> 4);
 #pragma unroll
                         for (int half = 0; half < 2; ++half) {
 #pragma unroll
-                            for (int k = 0; k < kTile / 16; ++k) {
-                                const uint64_t ad = sdesc_sw128(pa + k * 32, 16, 1024);
-                                const uint64_t bd = sdesc_sw128(vb + (4 * half) * kChunk + k * 2048, kChunk, 1024);
-                                mma_ss(tmem + 256 * half, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
-                            }
+                            for (int k = 0; k < kTile / 16; ++k)
+                                mma_ss(tmem + 256 * half, pd + 2 * k, vd + ((4 * half * kChunk + k * 2048) >> 4), idesc,
+                                       (first && k == 0) ? 0u : 1u);
                         }
-                        mma_commit(smem_u32(&bars[kBarVEmpty + st]));
+                        mma_commit(smem_u32(&bars[kOBarVEmpty + st]));
                         mma_commit(peer_pempty + 8 * pb);
                     }
                     __syncwarp();
                 }
                 if (!ok) break;
-                if (lane == 0) mma_commit(smem_u32(&bars[kBarOFull]));
+                if (lane == 0) mma_commit(smem_u32(&bars[kOBarOFull]));
                 __syncwarp();
                 ++kseg;
             }
             if (!ok && lane == 0) raise_abort(abort_flag, peer_abort, p.dev_status);
-            if (lane == 0) mma_commit(smem_u32(&bars[kBarFin]));
-            mbar_wait(&bars[kBarFin], 0, &never, kLimitNs);
-        } else {
+            if (lane == 0) {
+                mma_commit(smem_u32(&bars[kOBarFin]));
+                mbar_wait(&bars[kOBarFin], 0, &never, kLimitNs);
+            }
+            __syncwarp();
+        } else if (warp < 4) {
             // ---- epilogue: warps 0..3, one thread per query row
             const int r = tid;
             const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-            const float* alphas = reinterpret_cast<const float*>(smem + kOffAlpha);
             const int rr = g * kRows + r;
             const bool row_ok = rr < p.R;
             SegWalk w;
@@ -517,14 +609,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
                 for (;;) {
                     int ev = 0;  // 1: O complete, 2: rescale request, 3: give up
                     if (lane == 0) {
-                        if (mbar_test(smem_u32(&bars[kBarOFull]), kseg & 1u)) ev = 1;
-                        else if (mbar_test(smem_u32(&bars[kBarRescReq]), nresc & 1u)) ev = 2;
+                        if (mbar_test(smem_u32(&bars[kOBarOFull]), kseg & 1u)) ev = 1;
+                        else if (mbar_test(smem_u32(&bars[kOBarRescReq]), nresc & 1u)) ev = 2;
                         else if (*abort_flag) ev = 3;
                         else if ((++it & 255u) == 0 && globaltimer_ns() - t0 > kLimitNs) ev = 3;
                     }
                     ev = __shfl_sync(0xffffffffu, ev, 0);
                     if (ev == 1) {
-                        ok = mbar_wait(&bars[kBarOFull], kseg & 1u, abort_flag, kLimitNs);
+                        ok = mbar_wait(&bars[kOBarOFull], kseg & 1u, abort_flag, kLimitNs);
                         break;
                     }
                     if (ev == 3) {
@@ -532,11 +624,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
                         break;
                     }
                     if (ev == 2) {
-                        ok = mbar_wait(&bars[kBarRescReq], nresc & 1u, abort_flag, kLimitNs) &&
-                             mbar_wait(&bars[kBarODrain], nresc & 1u, abort_flag, kLimitNs);
+                        ok = mbar_wait(&bars[kOBarRescReq], nresc & 1u, abort_flag, kLimitNs) &&
+                             mbar_wait(&bars[kOBarODrain], nresc & 1u, abort_flag, kLimitNs);
                         __syncwarp();
                         tc_fence_after();
-                        const float a = alphas[*resc_pb * kRows + r];
+                        const float a =
+                            reinterpret_cast<const float*>(smem + kOOffMsg + *resc_pb * kMsgStride + kPBytes)[r];
                         if (__any_sync(0xffffffffu, a != 1.f)) {
 #pragma unroll 1
                             for (int c = 0; c < 16; ++c) {
@@ -550,7 +643,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
                             tmem_wait_st();
                         }
                         tc_fence_before();
-                        mbar_arrive(&bars[kBarRescDone]);
+                        mbar_arrive(&bars[kOBarRescDone]);
                         ++nresc;
                         if (!__all_sync(0xffffffffu, ok)) {
                             ok = false;
@@ -579,7 +672,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(&bars[kBarOFree]);
+                mbar_arrive(&bars[kOBarOFree]);
                 ++kseg;
             }
             if (!ok && lane == 0) raise_abort(abort_flag, peer_abort, p.dev_status);
@@ -590,7 +683,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const Params p) {
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // the peer no longer touches this CTA's shared memory
-    if (warp == 4) {
+    if (warp == kWarpProducer) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -654,15 +747,19 @@ cudaError_t launch_decode_tc(const uint16_t* q, const uint16_t* cache, int64_t c
         return cudaErrorNotSupported;
     auto encode = tc::encode_fn();
     if (!encode) return cudaErrorNotSupported;
-    CUtensorMap map;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(kRow), static_cast<cuuint64_t>(cap)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(kRow) * 2};
-    cuuint32_t box[2] = {64, 64};
-    cuuint32_t estr[2] = {1, 1};
-    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(cache), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+    // the cache as a 3-D tensor: (column within a 64-column chunk, token, chunk)
+    CUtensorMap maps[4];
+    const cuuint32_t nz[4] = {9, 6, 3, 8};
+    for (int i = 0; i < 4; ++i) {
+        cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(cap), 9};
+        cuuint64_t strides[2] = {static_cast<cuuint64_t>(kRow) * 2, 128};
+        cuuint32_t box[3] = {64, 64, nz[i]};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (encode(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(cache), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     tc::Params prm;
     prm.q = q;
     prm.seq_start = seq_start;
@@ -691,7 +788,7 @@ cudaError_t launch_decode_tc(const uint16_t* q, const uint16_t* cache, int64_t c
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel, map, prm);
+    return cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel, maps[0], maps[1], maps[2], maps[3], prm);
 }
 
 }  // namespace mla
