@@ -65,7 +65,7 @@ def step_counts(cfg: mi.MLAConfig, lengths: np.ndarray) -> dict:
     """Algorithmic bytes / FLOPs of one step (minimum traffic of the documented calls)."""
     H, T, n_q = cfg.H, cfg.T, cfg.n_q
     sum_L = int(lengths.sum())
-    cache = sum_L * mi.D_ROW * 2
+    cache = sum_L * mi.D_ROW * 2  # cached rows read (block padding is not counted)
     weights = 2 * H * mi.D_H * mi.D_C * 2
     q_in = T * H * (mi.D_H + mi.D_R) * 2
     q_abs = 2 * T * H * mi.D_ROW * 2            # written by absorb, read by attend
@@ -209,23 +209,27 @@ class Dist:
 
 def build_state(torch, mla, cfg: mi.MLAConfig, dev):
     lengths = mi.kv_lengths(cfg)
-    starts = mi.seq_starts(lengths)
+    starts = mi.seq_starts(lengths)  # rows of the generator's packed pool
     N = int(lengths.sum())
+    nblk = (lengths + mla.BLOCK_TOKENS - 1) // mla.BLOCK_TOKENS
+    seq_block = np.zeros(cfg.B, dtype=np.int64)
+    if cfg.B > 1:
+        seq_block[1:] = np.cumsum(nblk[:-1])
 
     def dbf(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
-    cache = torch.zeros((N, mi.D_ROW), dtype=torch.bfloat16, device=dev)
+    cache = torch.zeros((int(nblk.sum()), mla.BLOCK_BYTES), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     rope = mla.rope_table(int(lengths.max()), cfg.rope_base, dev)
-    seq_start = torch.from_numpy(starts).to(dev)
+    seq_block_t = torch.from_numpy(seq_block).to(dev)
     seq_of_row = np.repeat(np.arange(cfg.B, dtype=np.int32), lengths)
     pos_of_row = (np.arange(N, dtype=np.int64) - np.repeat(starts, lengths)).astype(np.int32)
     chunk = 1 << 18
     for r0 in range(0, N, chunk):
         n = min(chunk, N - r0)
         c, k = mi.token_rows(cfg, r0, n)
-        mla.append_cache(cache, seq_start, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
+        mla.append_cache(cache, seq_block_t, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
                          torch.from_numpy(pos_of_row[r0:r0 + n]).to(dev), dbf(c), dbf(k), rope, status)
     # the step's new tokens: the last n_q rows of every sequence
     new_rows = np.concatenate([starts[b] + lengths[b] - cfg.n_q + np.arange(cfg.n_q) for b in range(cfg.B)])
@@ -245,7 +249,7 @@ def build_state(torch, mla, cfg: mi.MLAConfig, dev):
     devt = {k: v.to(dev) for k, v in host.items()}
     T, H = cfg.T, cfg.H
     st = {
-        "lengths": lengths, "cache": cache, "status": status, "rope": rope, "seq_start": seq_start,
+        "lengths": lengths, "cache": cache, "status": status, "rope": rope, "seq_block": seq_block_t,
         "kv_len": torch.from_numpy(lengths.astype(np.int32)).to(dev),
         "W_UK": dbf(mi.weights(cfg, "uk")), "W_UV": dbf(mi.weights(cfg, "uv")),
         "host": host, "dev": devt,
@@ -262,17 +266,17 @@ def run_step(mla, cfg, st, ev=None):
     d = st["dev"]
     if ev:
         ev[0].record()
-    mla.append_cache(st["cache"], st["seq_start"], d["seq_idx"], d["pos"], d["c_kv"], d["k_rope"], st["rope"],
+    mla.append_cache(st["cache"], st["seq_block"], d["seq_idx"], d["pos"], d["c_kv"], d["k_rope"], st["rope"],
                      st["status"])
     mla.absorb_q(d["q_nope"], d["q_rope"], d["pos"], st["W_UK"], st["rope"], q_out=st["q_abs"],
                  dev_status=st["status"])
     if ev:
         ev[1].record()
-    mla.decode_attend(st["q_abs"], st["cache"], st["seq_start"], st["kv_len"], cfg.n_q, cfg.scale, 0, st["ws"],
+    mla.decode_attend(st["q_abs"], st["cache"], st["seq_block"], st["kv_len"], cfg.n_q, cfg.scale, 0, st["ws"],
                       dev_status=st["status"])
     if ev:
         ev[2].record()
-    mla.decode_finish(st["seq_start"], st["kv_len"], st["cache"], st["W_UV"], cfg.n_q, 0, st["ws"], st["out"])
+    mla.decode_finish(st["seq_block"], st["kv_len"], st["cache"], st["W_UV"], cfg.n_q, 0, st["ws"], st["out"])
     if ev:
         ev[3].record()
 

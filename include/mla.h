@@ -14,9 +14,20 @@
  *     RoPE with per-head q^R and one shared k^R; the RoPE'd key part is cached
  *     so keys need no rotation at inference; attention on [q^C; q^R].[k^C; k^R].
  *
- * Fixed sizes: d_c = 512, d_h^R = 64, d_h = 128 (packed cache row D = 576).
+ * Fixed sizes: d_c = 512, d_h^R = 64, d_h = 128 (cached row D = 576).
  * Runtime sizes: B sequences, H heads (1..128), n_q new query tokens per
  * sequence (1..16), T = B * n_q query rows (row t = b * n_q + j).
+ *
+ * Latent cache layout (blocked).  The cache is an array of blocks of
+ * MLA_BLOCK_TOKENS = 64 tokens, MLA_BLOCK_BYTES = 73728 bytes each.  Token
+ * `pos` of sequence b lives in block seq_block[b] + pos / 64, at row
+ * r = pos % 64; its 576 bf16 values [c^KV (0..511) | rotated k^R (512..575)]
+ * are stored as nine 64-column chunks, column c at byte offset
+ *     (c / 64) * 8192 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2
+ * within the block: each chunk is a [64 rows x 128 bytes] tile whose 16-byte
+ * units are permuted by the row index (the 128-byte swizzle), so that one
+ * contiguous copy places a block in shared memory exactly as the tensor-core
+ * operands are read.  Each sequence occupies ceil(L_b / 64) consecutive blocks.
  *
  * Conventions for every entry point:
  *   - All tensor arguments are DEVICE pointers to caller-owned memory, dense
@@ -49,6 +60,9 @@ extern "C" {
 
 typedef void* mla_stream; /* cudaStream_t */
 
+#define MLA_BLOCK_TOKENS 64
+#define MLA_BLOCK_BYTES 73728
+
 typedef enum {
     MLA_OK = 0,
     MLA_ERR_INVALID_ARG = 1,       /* null pointer, misalignment, negative size */
@@ -58,7 +72,7 @@ typedef enum {
 } mla_status;
 
 /* Bits a kernel ORs into *dev_status. */
-#define MLA_DEVERR_ROW_RANGE   0x1  /* a cache row outside [0, cap_tokens) was addressed */
+#define MLA_DEVERR_ROW_RANGE   0x1  /* a cache block outside [0, cap_blocks) was addressed */
 #define MLA_DEVERR_POS_RANGE   0x2  /* a position outside [0, rope_len) */
 #define MLA_DEVERR_KV_LEN      0x4  /* kv_len[b] < n_q */
 #define MLA_DEVERR_TIMEOUT     0x8  /* a bounded wait in a pipelined kernel expired */
@@ -92,11 +106,12 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* p
                         int T, int H, void* q_out, int32_t* dev_status, mla_stream stream);
 
 /*
- * mla_append_cache -- write T new tokens into the packed latent cache.
+ * mla_append_cache -- write T new tokens into the blocked latent cache.
  * ("两张账" page: only c^KV and k^R are cached; explainer 2.2.2: k^R is
  *  cached already rotated.)
- *   cache      bf16 [cap_tokens, 576]  row = seq_start[seq_idx[i]] + pos[i]
- *   seq_start  int64 [*]  first cache row of each sequence
+ *   cache      cap_blocks blocks of MLA_BLOCK_BYTES (layout above); token i
+ *              goes to block seq_block[seq_idx[i]] + pos[i] / 64, row pos[i] % 64
+ *   seq_block  int64 [*]  first cache block of each sequence
  *   seq_idx    int32 [T]  sequence of token i
  *   pos        int32 [T]  position of token i within its sequence
  *   c_kv       bf16 [T, 512]   copied to columns 0..511 bit for bit
@@ -106,7 +121,7 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* p
  * round-to-nearest-even to bf16: the result is reproducible bit for bit.
  * Out-of-range rows or positions set a MLA_DEVERR_* bit and are skipped.
  */
-mla_status mla_append_cache(void* cache, int64_t cap_tokens, const int64_t* seq_start,
+mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int64_t* seq_block,
                             const int32_t* seq_idx, const int32_t* pos, const void* c_kv,
                             const void* k_rope, const float* rope_table, int64_t rope_len,
                             int T, int32_t* dev_status, mla_stream stream);
@@ -128,10 +143,10 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
  *  latent space, W^UV afterwards; explainer 2.2.2 for the concatenated
  *  content/position inner product.)
  *   q          bf16 [B*n_q, H, 576]   from mla_absorb_q
- *   cache      bf16 [cap_tokens, 576] sequence b occupies rows
- *              seq_start[b] .. seq_start[b] + kv_len[b] - 1 (kv_len counts
- *              the n_q tokens of this step, already appended)
- *   seq_start  int64 [B];  kv_len int32 [B]
+ *   cache      cap_blocks blocks (layout above); sequence b occupies blocks
+ *              seq_block[b] .. seq_block[b] + ceil(kv_len[b] / 64) - 1 (kv_len
+ *              counts the n_q tokens of this step, already appended)
+ *   seq_block  int64 [B];  kv_len int32 [B]
  *   W_UV       bf16 [H, 128, 512]
  *   scale      softmax scale, 1/sqrt(d_h + d_h^R) = 1/sqrt(192) for V2 shapes
  *   num_splits 0: use every SM.  n > 0: at most n CTA pairs per group of 128
@@ -143,10 +158,10 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
  *   out        bf16 [B*n_q, H, 128]
  *   lse_out    fp32 [B*n_q, H] or NULL: log sum_t exp(s_t)
  * A sequence with kv_len[b] < n_q sets MLA_DEVERR_KV_LEN and its rows are
- * left unwritten; rows beyond cap_tokens set MLA_DEVERR_ROW_RANGE.
+ * left unwritten; blocks beyond cap_blocks set MLA_DEVERR_ROW_RANGE.
  */
-mla_status mla_decode(const void* q, const void* cache, int64_t cap_tokens,
-                      const int64_t* seq_start, const int32_t* kv_len, const void* W_UV,
+mla_status mla_decode(const void* q, const void* cache, int64_t cap_blocks,
+                      const int64_t* seq_block, const int32_t* kv_len, const void* W_UV,
                       int B, int n_q, int H, float scale, int num_splits,
                       void* workspace, size_t ws_bytes, void* out, float* lse_out,
                       int32_t* dev_status, mla_stream stream);
@@ -160,12 +175,12 @@ mla_status mla_decode(const void* q, const void* cache, int64_t cap_tokens,
  * same as for mla_decode; both calls must see the same sizes, num_splits and
  * workspace, and finish must be ordered after attend on the stream.
  */
-mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_tokens,
-                             const int64_t* seq_start, const int32_t* kv_len,
+mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_blocks,
+                             const int64_t* seq_block, const int32_t* kv_len,
                              int B, int n_q, int H, float scale, int num_splits,
                              void* workspace, size_t ws_bytes, int32_t* dev_status,
                              mla_stream stream);
-mla_status mla_decode_finish(const int64_t* seq_start, const int32_t* kv_len, int64_t cap_tokens,
+mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, int64_t cap_blocks,
                              const void* W_UV, int B, int n_q, int H, int num_splits,
                              void* workspace, size_t ws_bytes, void* out, float* lse_out,
                              mla_stream stream);
@@ -179,8 +194,8 @@ mla_status mla_decode_finish(const int64_t* seq_start, const int32_t* kv_len, in
  * mla_decode_cudacore_workspace_bytes().
  */
 size_t mla_decode_cudacore_workspace_bytes(int B, int n_q, int H, int num_splits);
-mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_tokens,
-                               const int64_t* seq_start, const int32_t* kv_len, const void* W_UV,
+mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_blocks,
+                               const int64_t* seq_block, const int32_t* kv_len, const void* W_UV,
                                int B, int n_q, int H, float scale, int num_splits,
                                void* workspace, size_t ws_bytes, void* out, float* lse_out,
                                int32_t* dev_status, mla_stream stream);

@@ -17,6 +17,8 @@ import torch
 
 D_C, D_R, D_H = 512, 64, 128
 D_ROW = D_C + D_R
+BLOCK_TOKENS = 64       # tokens per cache block
+BLOCK_BYTES = 73728     # 9 chunks x [64 rows x 128 bytes]
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_b200.so")
 if not os.path.exists(_LIB_PATH):
@@ -105,11 +107,22 @@ def absorb_q(q_nope, q_rope, pos, W_UK, rope_tab, q_out=None, dev_status=None, s
     return q_out
 
 
-def append_cache(cache, seq_start, seq_idx, pos, c_kv, k_rope, rope_tab, dev_status=None, stream=None):
-    """Write c_kv [T,512] and R_pos k_rope [T,64] into cache rows seq_start[seq_idx] + pos."""
+def new_cache(cap_blocks: int, device="cuda") -> torch.Tensor:
+    """An empty blocked latent cache: uint8 [cap_blocks, BLOCK_BYTES] (layout in include/mla.h)."""
+    return torch.empty((cap_blocks, BLOCK_BYTES), dtype=torch.uint8, device=device)
+
+
+def _cache_ptr(cache):
+    if cache.dim() != 2 or cache.shape[1] != BLOCK_BYTES:
+        raise MLAError(f"cache must be uint8 [cap_blocks, {BLOCK_BYTES}]")
+    return _ptr(cache, torch.uint8, None, "cache")
+
+
+def append_cache(cache, seq_block, seq_idx, pos, c_kv, k_rope, rope_tab, dev_status=None, stream=None):
+    """Write c_kv [T,512] and R_pos k_rope [T,64] at token pos of sequence seq_idx (block seq_block[seq_idx] + pos/64)."""
     T = c_kv.shape[0]
     _check(lib.mla_append_cache(
-        _ptr(cache, torch.bfloat16, None, "cache"), cache.shape[0], _ptr(seq_start, torch.int64, None, "seq_start"),
+        _cache_ptr(cache), cache.shape[0], _ptr(seq_block, torch.int64, None, "seq_block"),
         _ptr(seq_idx, torch.int32, (T,), "seq_idx"), _ptr(pos, torch.int32, (T,), "pos"),
         _ptr(c_kv, torch.bfloat16, (T, D_C), "c_kv"), _ptr(k_rope, torch.bfloat16, (T, D_R), "k_rope"),
         _ptr(rope_tab, torch.float32, None, "rope_table"), rope_tab.shape[0], T,
@@ -120,7 +133,7 @@ def decode_workspace_bytes(B: int, n_q: int, H: int, num_splits: int = 0) -> int
     return int(lib.mla_decode_workspace_bytes(B, n_q, H, num_splits))
 
 
-def decode(q, cache, seq_start, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
+def decode(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
            workspace=None, out=None, lse_out=None, dev_status=None, stream=None):
     """One absorbed decode step: out bf16 [B*n_q, H, 128] (and lse fp32 [B*n_q, H] if given)."""
     B = kv_len.shape[0]
@@ -133,8 +146,8 @@ def decode(q, cache, seq_start, kv_len, W_UV, n_q: int, scale: float, num_splits
     if out is None:
         out = torch.empty((T, H, D_H), dtype=torch.bfloat16, device=q.device)
     _check(lib.mla_decode(
-        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _ptr(cache, torch.bfloat16, None, "cache"), cache.shape[0],
-        _ptr(seq_start, torch.int64, (B,), "seq_start"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0],
+        _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, float(scale), num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(out, torch.bfloat16, (T, H, D_H), "out"), _ptr(lse_out, torch.float32, (T, H), "lse_out"),
@@ -142,26 +155,26 @@ def decode(q, cache, seq_start, kv_len, W_UV, n_q: int, scale: float, num_splits
     return out
 
 
-def decode_attend(q, cache, seq_start, kv_len, n_q: int, scale: float, num_splits: int, workspace,
+def decode_attend(q, cache, seq_block, kv_len, n_q: int, scale: float, num_splits: int, workspace,
                   dev_status=None, stream=None):
     """Phase 1 of decode: per-split partials into ``workspace``."""
     B = kv_len.shape[0]
     T, H = q.shape[0], q.shape[1]
     _check(lib.mla_decode_attend(
-        _ptr(q, torch.bfloat16, (B * n_q, H, D_ROW), "q"), _ptr(cache, torch.bfloat16, None, "cache"),
-        cache.shape[0], _ptr(seq_start, torch.int64, (B,), "seq_start"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        _ptr(q, torch.bfloat16, (B * n_q, H, D_ROW), "q"), _cache_ptr(cache),
+        cache.shape[0], _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
         B, n_q, H, float(scale), num_splits, _ptr(workspace, None, None, "workspace"),
         workspace.numel() * workspace.element_size(), _ptr(dev_status, torch.int32, None, "dev_status"),
         _stream(stream)))
 
 
-def decode_finish(seq_start, kv_len, cache, W_UV, n_q: int, num_splits: int, workspace, out, lse_out=None,
+def decode_finish(seq_block, kv_len, cache, W_UV, n_q: int, num_splits: int, workspace, out, lse_out=None,
                   stream=None):
     """Phase 2 of decode: merge the partials, apply W^UV into ``out`` bf16 [B*n_q, H, 128]."""
     B = kv_len.shape[0]
     H = W_UV.shape[0]
     _check(lib.mla_decode_finish(
-        _ptr(seq_start, torch.int64, (B,), "seq_start"), _ptr(kv_len, torch.int32, (B,), "kv_len"), cache.shape[0],
+        _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"), cache.shape[0],
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(out, torch.bfloat16, (B * n_q, H, D_H), "out"), _ptr(lse_out, torch.float32, (B * n_q, H), "lse_out"),
@@ -169,7 +182,7 @@ def decode_finish(seq_start, kv_len, cache, W_UV, n_q: int, num_splits: int, wor
     return out
 
 
-def decode_cudacore(q, cache, seq_start, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
+def decode_cudacore(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
                     workspace=None, out=None, lse_out=None, dev_status=None, stream=None):
     """The decode step on CUDA cores (second implementation, same results within fp32 rounding)."""
     B = kv_len.shape[0]
@@ -182,8 +195,8 @@ def decode_cudacore(q, cache, seq_start, kv_len, W_UV, n_q: int, scale: float, n
     if out is None:
         out = torch.empty((T, H, D_H), dtype=torch.bfloat16, device=q.device)
     _check(lib.mla_decode_cudacore(
-        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _ptr(cache, torch.bfloat16, None, "cache"), cache.shape[0],
-        _ptr(seq_start, torch.int64, (B,), "seq_start"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0],
+        _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, float(scale), num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(out, torch.bfloat16, (T, H, D_H), "out"), _ptr(lse_out, torch.float32, (T, H), "lse_out"),

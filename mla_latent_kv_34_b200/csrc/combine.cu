@@ -108,18 +108,19 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int T, in
 // The segments of sequence b are the pieces of the equal cluster ranges
 // [p Nt / P, (p+1) Nt / P) of the global tile space that overlap its tiles.
 
-__device__ __forceinline__ int tc_seq_tiles(const int32_t* kv_len, const int64_t* seq_start, int64_t cap, int n_q,
-                                            int b) {
+__device__ __forceinline__ int tc_seq_tiles(const int32_t* kv_len, const int64_t* seq_block, int64_t cap_blocks,
+                                            int n_q, int b) {
     const int L = kv_len[b];
     if (L < n_q) return 0;
-    const int64_t s = seq_start[b];
-    if (s < 0 || s + L > cap) return 0;
-    return (L + 63) / 64;
+    const int64_t s = seq_block[b];
+    const int nt = (L + kBlockTokens - 1) / kBlockTokens;
+    if (s < 0 || s + nt > cap_blocks) return 0;
+    return nt;
 }
 
 __global__ void __launch_bounds__(256) combine_tc_kernel(
     const float* __restrict__ o_part, const float2* __restrict__ ml_part, const int32_t* __restrict__ kv_len,
-    const int64_t* __restrict__ seq_start, int64_t cap, int B, int n_q, int H, int P_g, int slots,
+    const int64_t* __restrict__ seq_block, int64_t cap_blocks, int B, int n_q, int H, int P_g, int slots,
     const uint16_t* __restrict__ W_UV, uint16_t* __restrict__ out, float* __restrict__ lse_out) {
     __shared__ float ol[kCombTok][kDc];
     __shared__ int red[2][8];
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(256) combine_tc_kernel(
     // total tiles and tiles before b_lo
     int s_all = 0, s_before = 0;
     for (int b = tid; b < B; b += blockDim.x) {
-        const int v = tc_seq_tiles(kv_len, seq_start, cap, n_q, b);
+        const int v = tc_seq_tiles(kv_len, seq_block, cap_blocks, n_q, b);
         s_all += v;
         s_before += (b < b_lo) ? v : 0;
     }
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(256) combine_tc_kernel(
         red[0][0] = a;
         int ts = bb;
         for (int b = b_lo; b <= b_hi; ++b) {
-            const int v = tc_seq_tiles(kv_len, seq_start, cap, n_q, b);
+            const int v = tc_seq_tiles(kv_len, seq_block, cap_blocks, n_q, b);
             ts_of[b - b_lo] = ts;
             nt_of[b - b_lo] = v;
             ts += v;
@@ -209,11 +210,11 @@ __global__ void __launch_bounds__(256) combine_tc_kernel(
 }
 
 cudaError_t launch_combine_tc(const float* o_part, const float2* ml_part, const int32_t* kv_len,
-                              const int64_t* seq_start, int64_t cap, int B, int n_q, int H, int P_g, int slots,
+                              const int64_t* seq_block, int64_t cap_blocks, int B, int n_q, int H, int P_g, int slots,
                               const uint16_t* W_UV, uint16_t* out, float* lse_out, cudaStream_t stream) {
     const int T = B * n_q;
     dim3 grid(H, (T + kCombTok - 1) / kCombTok);
-    combine_tc_kernel<<<grid, 256, 0, stream>>>(o_part, ml_part, kv_len, seq_start, cap, B, n_q, H, P_g, slots, W_UV,
+    combine_tc_kernel<<<grid, 256, 0, stream>>>(o_part, ml_part, kv_len, seq_block, cap_blocks, B, n_q, H, P_g, slots, W_UV,
                                                 out, lse_out);
     return cudaGetLastError();
 }

@@ -39,8 +39,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 __global__ void __launch_bounds__(256) decode_simt_kernel(
-    const uint16_t* __restrict__ q, const uint16_t* __restrict__ cache, int64_t cap,
-    const int64_t* __restrict__ seq_start, const int32_t* __restrict__ kv_len, int n_q, int H,
+    const uint16_t* __restrict__ q, const uint8_t* __restrict__ cache, int64_t cap_blocks,
+    const int64_t* __restrict__ seq_block, const int32_t* __restrict__ kv_len, int n_q, int H,
     float scale_log2, int S, float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* dev_status) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem& sm = *reinterpret_cast<SimtSmem*>(smem_raw);
@@ -51,12 +51,12 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
     const int nrows = min(kSimtRows, R - r0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int L = kv_len[b];
-    const int64_t start = seq_start[b];
+    const int64_t blk0 = seq_block[b];
     if (L < n_q) {
         if (tid == 0 && s == 0 && blockIdx.y == 0) report(dev_status, MLA_DEVERR_KV_LEN);
         return;
     }
-    if (start < 0 || start + L > cap) {
+    if (blk0 < 0 || blk0 + (L + kBlockTokens - 1) / kBlockTokens > cap_blocks) {
         if (tid == 0 && s == 0 && blockIdx.y == 0) report(dev_status, MLA_DEVERR_ROW_RANGE);
         return;
     }
@@ -83,13 +83,15 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
 #pragma unroll
     for (int r = 0; r < kSimtRows; ++r) acc[r][0] = acc[r][1] = 0.f;
 
-    const uint32_t* cache32 = reinterpret_cast<const uint32_t*>(cache);
     for (int ts = t_lo; ts < t_hi; ts += kSimtTok) {
         __syncthreads();
         for (int idx = tid; idx < kSimtTok * (kRow / 2); idx += blockDim.x) {
             const int tk = idx / (kRow / 2), w = idx % (kRow / 2);
             const int t = ts + tk;
-            sm.kv[tk][w] = (t < t_hi) ? cache32[(start + t) * (kRow / 2) + w] : 0u;
+            sm.kv[tk][w] = (t < t_hi) ? *reinterpret_cast<const uint32_t*>(
+                                            cache + (blk0 + t / kBlockTokens) * kBlockBytes +
+                                            block_offset(t % kBlockTokens, 2 * w))
+                                      : 0u;
         }
         __syncthreads();
         // scores: lane = token, two rows per warp
@@ -154,7 +156,7 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
     }
 }
 
-cudaError_t launch_decode_simt(const uint16_t* q, const uint16_t* cache, int64_t cap, const int64_t* seq_start,
+cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
                                const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,
                                float* o_part, float* lse_part, int32_t* dev_status, cudaStream_t stream) {
     const int R = n_q * H;
@@ -164,7 +166,7 @@ cudaError_t launch_decode_simt(const uint16_t* q, const uint16_t* cache, int64_t
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const float scale_log2 = scale * 1.44269504088896340736f;
-    decode_simt_kernel<<<grid, 256, smem, stream>>>(q, cache, cap, seq_start, kv_len, n_q, H, scale_log2, splits,
+    decode_simt_kernel<<<grid, 256, smem, stream>>>(q, cache, cap_blocks, seq_block, kv_len, n_q, H, scale_log2, splits,
                                                     o_part, lse_part, dev_status);
     return cudaGetLastError();
 }

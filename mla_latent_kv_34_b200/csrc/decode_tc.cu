@@ -8,16 +8,17 @@
 //
 // Work split.  A cluster of two CTAs (one SM each) owns 128 query rows:
 //   CTA 0 ("S"): the 128 absorbed query rows live in TMEM (the A operand, 288
-//     columns); each 64-token tile of the cache is TMA-loaded (9 swizzled
-//     [64 x 64] chunks) and S = Q K^T is formed by 36 tcgen05.mma (M=128,
+//     columns); each 64-token block of the cache (9 pre-swizzled [64 x 64]
+//     chunks, 72 KB contiguous) arrives with one bulk copy into a ring of
+//     chunk slots, and S = Q K^T is formed by 36 tcgen05.mma (M=128,
 //     N=64, K=16) into one of two TMEM score buffers.  Eight warps (a query
 //     row's 64 scores split over two threads) run the online softmax in fp32,
 //     stage P (bf16) in shared memory, and one thread ships each P tile to
 //     CTA 1 with a single asynchronous bulk copy over DSMEM.
 //   CTA 1 ("O"): keeps the unnormalised latent output O[128 x 512] fp32 in its
 //     whole TMEM and accumulates O += P V with 8 tcgen05.mma (M=128, N=256,
-//     K=16) per tile; V is the first 512 columns of the same cache tile, read
-//     as an MN-major operand.
+//     K=16) per tile; V is the first 512 columns of the same cache block (its
+//     first 64 KB, one bulk copy), read as an MN-major operand.
 // O for 128 rows x 512 fp32 fills an SM's 256 KB of TMEM, hence the pair.
 //
 // The softmax keeps a stale running max: it only rescales when a tile's max
@@ -35,7 +36,6 @@
 // both CTAs of the pair abandon their loops, let in-flight copies and MMAs
 // land, free TMEM and return.
 #include <cuda.h>
-#include <cudaTypedefs.h>
 #include <math_constants.h>
 
 #include "mla_internal.cuh"
@@ -74,10 +74,12 @@ constexpr int kSOffRing = 0;                                  // 24 x 8 KB
 constexpr int kSOffStage = kRing * kChunk;                    // 2 x kMsgBytes (local P messages)
 constexpr int kSOffXchg = kSOffStage + 2 * kMsgBytes;         // [2][128] fp32 half-row maxima / sums
 constexpr int kSOffBar = kSOffXchg + 2 * kRows * 4;
-// barrier slots, S CTA: a tile's chunks arrive together (one or two TMA boxes) on
-// kSBarTFull[tile % 3]; ring slots are released one chunk at a time.
+// barrier slots, S CTA: a tile's chunks arrive together (one or two bulk copies) on
+// kSBarTFull[tile % 3]; the ring is released in triples of chunks (a tile always
+// starts on a triple: 9 n mod 24 is a multiple of 3), three commits per tile.
 constexpr int kTilesInRing = 3;  // at most 3 tiles own ring slots at any time (24 / 9 rounded up)
-constexpr int kSBarTFull = 0, kSBarEmpty = kTilesInRing, kSBarSFull = kSBarEmpty + kRing,
+constexpr int kTriples = kRing / 3;
+constexpr int kSBarTFull = 0, kSBarEmpty = kTilesInRing, kSBarSFull = kSBarEmpty + kTriples,
               kSBarSEmpty = kSBarSFull + 2, kSBarPEmpty = kSBarSEmpty + 2, kSBarQReady = kSBarPEmpty + 2,
               kSBarFin = kSBarQReady + 1, kSNumBars = kSBarFin + 1;
 constexpr int kSOffTail = kSOffBar + kSNumBars * 8;
@@ -97,12 +99,13 @@ static_assert(kOOffMsg % 1024 == 0 && kMsgStride % 1024 == 0, "P tiles must be 1
 
 struct Params {
     const uint16_t* q;
-    const int64_t* seq_start;
+    const uint8_t* cache;  // blocks of kBlockBytes
+    const int64_t* seq_block;
     const int32_t* kv_len;
     float* o_part;    // [G][slots][128][512]
     float2* ml_part;  // [G][slots][128]  (running max in log2 units, sum)
     int32_t* dev_status;
-    int64_t cap;
+    int64_t cap_blocks;
     int B, n_q, H, R, G, P_g, slots;
     float scale_log2;
 };
@@ -110,14 +113,15 @@ struct Params {
 __device__ __forceinline__ int seq_tiles(const Params& p, int b) {
     const int L = p.kv_len[b];
     if (L < p.n_q) return 0;
-    const int64_t s = p.seq_start[b];
-    if (s < 0 || s + L > p.cap) return 0;
-    return (L + kTile - 1) / kTile;
+    const int64_t s = p.seq_block[b];
+    const int nt = (L + kTile - 1) / kTile;
+    if (s < 0 || s + nt > p.cap_blocks) return 0;
+    return nt;
 }
 
 struct Seg {
     int b, t0, t1, L, slot;
-    int64_t row0;
+    int64_t blk0;  // first cache block of the sequence
 };
 
 // Walks the segments of one cluster's tile range [lo, hi).
@@ -148,7 +152,7 @@ struct SegWalk {
                 s.t0 = a - ctb;
                 s.t1 = e - ctb;
                 s.L = p.kv_len[cb];
-                s.row0 = p.seq_start[cb];
+                s.blk0 = p.seq_block[cb];
                 s.slot = cb + pidx;
                 return true;
             }
@@ -176,8 +180,7 @@ __device__ __forceinline__ float fmax32(const float (&v)[32]) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant__ CUtensorMap kv6,
-                 const __grid_constant__ CUtensorMap kv3, const __grid_constant__ CUtensorMap v8, const Params p) {
+decode_tc_kernel(const Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -198,7 +201,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
     if (tid == 0) {
         if (rank == 0) {
             for (int i = 0; i < kTilesInRing; ++i) mbar_init(&bars[kSBarTFull + i], 1);
-            for (int i = 0; i < kRing; ++i) mbar_init(&bars[kSBarEmpty + i], 1);
+            for (int i = 0; i < kTriples; ++i) mbar_init(&bars[kSBarEmpty + i], 1);
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&bars[kSBarSFull + i], 1);
                 mbar_init(&bars[kSBarSEmpty + i], kSoftThreads);
@@ -231,7 +234,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
             if (blockIdx.x == 0 && p.dev_status) {
                 const int L = p.kv_len[b];
                 if (L < p.n_q) atomicOr(p.dev_status, MLA_DEVERR_KV_LEN);
-                else if (p.seq_start[b] < 0 || p.seq_start[b] + L > p.cap) atomicOr(p.dev_status, MLA_DEVERR_ROW_RANGE);
+                else if (p.seq_block[b] < 0 || p.seq_block[b] + (L + kTile - 1) / kTile > p.cap_blocks)
+                    atomicOr(p.dev_status, MLA_DEVERR_ROW_RANGE);
             }
         }
 #pragma unroll
@@ -256,14 +260,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
     if (active && rank == 0) {
         // =============================================================== S CTA
         if (warp == kWarpProducer) {
-            // ---- TMA producer.  The cache is viewed as a 3-D tensor (column in chunk, token,
-            //      chunk) so that one box lands a whole 64-token tile chunk-major in the
-            //      24-slot ring (a tile that wraps the ring end takes two boxes: 6 + 3 or
-            //      3 + 6 chunks).  A second walker pulls tiles kPrefetchTiles ahead into L2.
+            // ---- copy producer: each 64-token block (72 KB, already in the operand layout)
+            //      lands in the 24-slot ring with one bulk copy (two when it wraps the ring
+            //      end: 6 + 3 or 3 + 6 chunks).  A second walker pulls blocks kPrefetchTiles
+            //      ahead into L2.
             if (lane == 0) {
-                prefetch_tmap(&kv9);
-                prefetch_tmap(&kv6);
-                prefetch_tmap(&kv3);
                 SegWalk w, wp;
                 w.init(p, lo, hi, pidx);
                 wp.init(p, lo, hi, pidx);
@@ -272,7 +273,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
                 int tp = have_p ? sp.t0 : 0;
                 auto prefetch_one = [&]() {
                     if (!have_p) return;
-                    tma_prefetch_3d(&kv9, 0, static_cast<int>(sp.row0 + static_cast<int64_t>(tp) * kTile), 0);
+                    bulk_prefetch_l2(p.cache + (sp.blk0 + tp) * kBlockBytes, kBlockBytes);
                     if (++tp >= sp.t1) {
                         have_p = wp.next(p, sp);
                         tp = have_p ? sp.t0 : 0;
@@ -285,21 +286,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
                     for (int t = s.t0; ok && t < s.t1; ++t, ++n) {
                         prefetch_one();
                         const uint32_t gc = n * kKvChunks, s0 = gc % kRing;
-                        for (int c = 0; ok && c < kKvChunks; ++c) {
-                            const uint32_t g2 = gc + c;
-                            ok = mbar_wait(&bars[kSBarEmpty + g2 % kRing], ((g2 / kRing) & 1u) ^ 1u, abort_flag, kLimitNs);
+                        for (int c = 0; ok && c < 3; ++c) {
+                            const uint32_t g3 = gc / 3 + c;  // triple counter
+                            ok = mbar_wait(&bars[kSBarEmpty + g3 % kTriples], ((g3 / kTriples) & 1u) ^ 1u, abort_flag,
+                                           kLimitNs);
                         }
                         if (!ok) break;
                         uint64_t* tb = &bars[kSBarTFull + n % kTilesInRing];
                         mbar_arrive_expect_tx(tb, kKvChunks * kChunk);
-                        const int y = static_cast<int>(s.row0 + static_cast<int64_t>(t) * kTile);
+                        const uint8_t* src = p.cache + (s.blk0 + t) * kBlockBytes;
                         const uint32_t dst = sbase + kSOffRing + s0 * kChunk;
                         if (s0 + kKvChunks <= static_cast<uint32_t>(kRing)) {
-                            tma_load_3d(dst, &kv9, 0, y, 0, tb);
+                            bulk_load(dst, src, kKvChunks * kChunk, tb);
                         } else {
-                            const uint32_t first = kRing - s0;  // 6 or 3 chunks up to the ring end
-                            tma_load_3d(dst, first == 6 ? &kv6 : &kv3, 0, y, 0, tb);
-                            tma_load_3d(sbase + kSOffRing, first == 6 ? &kv3 : &kv6, 0, y, static_cast<int>(first), tb);
+                            const uint32_t first = kRing - s0;  // chunks up to the ring end
+                            bulk_load(dst, src, first * kChunk, tb);
+                            bulk_load(sbase + kSOffRing, src + first * kChunk, (kKvChunks - first) * kChunk, tb);
                         }
                     }
                 }
@@ -311,7 +313,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
         } else if (warp == kWarpMma) {
             // ---- MMA issuer (one thread): S[sb] = Q K^T, A from TMEM, B = cache chunks
             //      (K-major SW128).  Once a tile has landed its 36 MMAs go out back to back;
-            //      each chunk's ring slot is released (commit) as soon as its 4 MMAs finish.
+            //      each triple of ring slots is released (commit) once its 12 MMAs finish.
             if (lane == 0) {
                 constexpr uint32_t idesc = idesc_bf16_f32(kRows, kTile, false, false);
                 const uint64_t ring_desc = sdesc_sw128(sbase + kSOffRing, 16, 1024);
@@ -331,14 +333,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t d = tmem + col_s(sb);
+                        const uint32_t s0 = gc % kRing;
 #pragma unroll
                         for (int c = 0; c < kKvChunks; ++c) {
-                            const uint32_t slot = (gc + c) % kRing;
-                            const uint64_t cd = ring_desc + (static_cast<uint64_t>(slot * kChunk) >> 4);
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                mma_ts(d, tmem + kColQ + 8 * (4 * c + k), cd + 2 * k, idesc, (c | k) ? 1u : 0u);
-                            mma_commit(smem_u32(&bars[kSBarEmpty + slot]));  // slot free once these 4 finish
+                            const uint32_t slot = (s0 + c) % kRing;
+                            const uint64_t cd = ring_desc + (static_cast<uint64_t>(slot) << 9);  // 8 KB / 16
+                            const uint32_t qa = tmem + kColQ + 32 * c;
+                            mma_ts(d, qa, cd, idesc, c ? 1u : 0u);
+                            mma_ts(d, qa + 8, cd + 2, idesc, 1u);
+                            mma_ts(d, qa + 16, cd + 4, idesc, 1u);
+                            mma_ts(d, qa + 24, cd + 6, idesc, 1u);
+                            if (c % 3 == 2)  // triple free once its 12 MMAs finish
+                                mma_commit(smem_u32(&bars[kSBarEmpty + ((gc / 3 + c / 3) % kTriples)]));
                         }
                         mma_commit(smem_u32(&bars[kSBarSFull + sb]));
                     }
@@ -491,9 +497,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
     } else if (active && rank == 1) {
         // =============================================================== O CTA
         if (warp == kWarpProducer) {
-            // ---- TMA producer: the 8 latent chunks of each tile (V)
+            // ---- copy producer: the 8 latent chunks of each block (its first 64 KB) = V
             if (lane == 0) {
-                prefetch_tmap(&v8);
                 SegWalk w;
                 w.init(p, lo, hi, pidx);
                 Seg s;
@@ -507,8 +512,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
                             break;
                         }
                         mbar_arrive_expect_tx(&bars[kOBarVFull + st], kVChunks * kChunk);
-                        const int y = static_cast<int>(s.row0 + static_cast<int64_t>(t) * kTile);
-                        tma_load_3d(sbase + kOOffV + st * kVChunks * kChunk, &v8, 0, y, 0, &bars[kOBarVFull + st]);
+                        bulk_load(sbase + kOOffV + st * kVChunks * kChunk, p.cache + (s.blk0 + t) * kBlockBytes,
+                                  kVChunks * kChunk, &bars[kOBarVFull + st]);
                     }
                 }
                 if (!ok) raise_abort(abort_flag, peer_abort, p.dev_status);
@@ -651,7 +656,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
                         }
                         continue;
                     }
-                    __nanosleep(64);
+                    __nanosleep(256);
                 }
                 ok = __all_sync(0xffffffffu, ok);
                 __syncwarp();
@@ -689,18 +694,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kv9, const __grid_constant_
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 }  // namespace tc
 
 int decode_tc_max_clusters() { return 74; }
@@ -731,7 +724,7 @@ int decode_tc_clusters() {
     return cache[dev];
 }
 
-cudaError_t launch_decode_tc(const uint16_t* q, const uint16_t* cache, int64_t cap, const int64_t* seq_start,
+cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
                              const int32_t* kv_len, int B, int n_q, int H, float scale, int clusters_per_group,
                              float* o_part, float2* ml_part, int slots, int32_t* dev_status, cudaStream_t stream) {
     const int R = n_q * H;
@@ -745,29 +738,15 @@ cudaError_t launch_decode_tc(const uint16_t* q, const uint16_t* cache, int64_t c
     if (cudaFuncSetAttribute(tc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::kSmemBytes) !=
         cudaSuccess)
         return cudaErrorNotSupported;
-    auto encode = tc::encode_fn();
-    if (!encode) return cudaErrorNotSupported;
-    // the cache as a 3-D tensor: (column within a 64-column chunk, token, chunk)
-    CUtensorMap maps[4];
-    const cuuint32_t nz[4] = {9, 6, 3, 8};
-    for (int i = 0; i < 4; ++i) {
-        cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(cap), 9};
-        cuuint64_t strides[2] = {static_cast<cuuint64_t>(kRow) * 2, 128};
-        cuuint32_t box[3] = {64, 64, nz[i]};
-        cuuint32_t estr[3] = {1, 1, 1};
-        if (encode(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(cache), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return cudaErrorInvalidValue;
-    }
     tc::Params prm;
     prm.q = q;
-    prm.seq_start = seq_start;
+    prm.cache = cache;
+    prm.seq_block = seq_block;
     prm.kv_len = kv_len;
     prm.o_part = o_part;
     prm.ml_part = ml_part;
     prm.dev_status = dev_status;
-    prm.cap = cap;
+    prm.cap_blocks = cap_blocks;
     prm.B = B;
     prm.n_q = n_q;
     prm.H = H;
@@ -788,7 +767,7 @@ cudaError_t launch_decode_tc(const uint16_t* q, const uint16_t* cache, int64_t c
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel, maps[0], maps[1], maps[2], maps[3], prm);
+    return cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel, prm);
 }
 
 }  // namespace mla

@@ -60,8 +60,8 @@ int tc_clusters_per_group(int G, int num_splits) {
     return pg;
 }
 
-mla_status check_decode_shape(int B, int64_t cap_tokens, int n_q, int H, int num_splits) {
-    if (B < 0 || cap_tokens < 0 || cap_tokens >= (int64_t(1) << 31)) return MLA_ERR_INVALID_ARG;
+mla_status check_decode_shape(int B, int64_t cap_blocks, int n_q, int H, int num_splits) {
+    if (B < 0 || cap_blocks < 0 || cap_blocks >= (int64_t(1) << 31) / kBlockTokens) return MLA_ERR_INVALID_ARG;
     if (H < 1 || H > kMaxHeads || n_q < 1 || n_q > kMaxNq || num_splits < 0 || num_splits > 256)
         return MLA_ERR_UNSUPPORTED_SHAPE;
     return MLA_OK;
@@ -76,7 +76,7 @@ int mla_abi_version(void) { return 1; }
 const char* mla_status_string(int status) {
     switch (status) {
         case MLA_OK: return "ok";
-        case MLA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, negative size)";
+        case MLA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, negative or too large size)";
         case MLA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (H in 1..128, n_q in 1..16, splits in 0..256)";
         case MLA_ERR_CUDA: return "CUDA runtime error";
         case MLA_ERR_WORKSPACE: return "workspace too small";
@@ -87,7 +87,7 @@ const char* mla_status_string(int status) {
 const char* mla_device_status_string(int32_t w) {
     if (w == 0) return "ok";
     if (w & MLA_DEVERR_TIMEOUT) return "bounded wait expired in a pipelined kernel";
-    if (w & MLA_DEVERR_ROW_RANGE) return "cache row outside [0, cap_tokens)";
+    if (w & MLA_DEVERR_ROW_RANGE) return "cache block outside [0, cap_blocks)";
     if (w & MLA_DEVERR_POS_RANGE) return "position outside the RoPE table";
     if (w & MLA_DEVERR_KV_LEN) return "kv_len smaller than n_q";
     return "unknown device error bits";
@@ -121,15 +121,15 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* p
                                        static_cast<cudaStream_t>(stream)));
 }
 
-mla_status mla_append_cache(void* cache, int64_t cap_tokens, const int64_t* seq_start, const int32_t* seq_idx,
+mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int64_t* seq_block, const int32_t* seq_idx,
                             const int32_t* pos, const void* c_kv, const void* k_rope, const float* rope_table,
                             int64_t rope_len, int T, int32_t* dev_status, mla_stream stream) {
-    if (T < 0 || cap_tokens < 0 || rope_len < 0) return MLA_ERR_INVALID_ARG;
+    if (T < 0 || cap_blocks < 0 || rope_len < 0) return MLA_ERR_INVALID_ARG;
     if (T == 0) return MLA_OK;
-    if (!cache || !seq_start || !seq_idx || !pos || !c_kv || !k_rope || !rope_table) return MLA_ERR_INVALID_ARG;
+    if (!cache || !seq_block || !seq_idx || !pos || !c_kv || !k_rope || !rope_table) return MLA_ERR_INVALID_ARG;
     if (!aligned16(cache) || !aligned16(c_kv) || !aligned16(k_rope) || !aligned16(rope_table))
         return MLA_ERR_INVALID_ARG;
-    return cuda_status(launch_append_cache(static_cast<uint16_t*>(cache), cap_tokens, seq_start, seq_idx, pos,
+    return cuda_status(launch_append_cache(static_cast<uint8_t*>(cache), cap_blocks, seq_block, seq_idx, pos,
                                            static_cast<const uint16_t*>(c_kv), static_cast<const uint16_t*>(k_rope),
                                            rope_table, rope_len, T, dev_status, static_cast<cudaStream_t>(stream)));
 }
@@ -139,34 +139,34 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits) {
     return tc_ws_layout(B, n_q, H).total;
 }
 
-mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_tokens, const int64_t* seq_start,
+mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_blocks, const int64_t* seq_block,
                              const int32_t* kv_len, int B, int n_q, int H, float scale, int num_splits,
                              void* workspace, size_t ws_bytes, int32_t* dev_status, mla_stream stream) {
-    mla_status st = check_decode_shape(B, cap_tokens, n_q, H, num_splits);
+    mla_status st = check_decode_shape(B, cap_blocks, n_q, H, num_splits);
     if (st != MLA_OK) return st;
     if (!(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
     if (B == 0) return MLA_OK;
-    if (!q || !cache || !seq_start || !kv_len || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!q || !cache || !seq_block || !kv_len || !workspace) return MLA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(cache) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
     const TcWs lay = tc_ws_layout(B, n_q, H);
     if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
     const int pg = tc_clusters_per_group(lay.G, num_splits);
     if (pg <= 0) return MLA_ERR_CUDA;
     char* ws = static_cast<char*>(workspace);
-    return cuda_status(launch_decode_tc(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(cache),
-                                        cap_tokens, seq_start, kv_len, B, n_q, H, scale, pg,
+    return cuda_status(launch_decode_tc(static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(cache),
+                                        cap_blocks, seq_block, kv_len, B, n_q, H, scale, pg,
                                         reinterpret_cast<float*>(ws + lay.o_part),
                                         reinterpret_cast<float2*>(ws + lay.ml_part), lay.slots, dev_status,
                                         static_cast<cudaStream_t>(stream)));
 }
 
-mla_status mla_decode_finish(const int64_t* seq_start, const int32_t* kv_len, int64_t cap_tokens, const void* W_UV,
+mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, int64_t cap_blocks, const void* W_UV,
                              int B, int n_q, int H, int num_splits, void* workspace, size_t ws_bytes, void* out,
                              float* lse_out, mla_stream stream) {
-    mla_status st = check_decode_shape(B, cap_tokens, n_q, H, num_splits);
+    mla_status st = check_decode_shape(B, cap_blocks, n_q, H, num_splits);
     if (st != MLA_OK) return st;
     if (B == 0) return MLA_OK;
-    if (!seq_start || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!seq_block || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
     if (!aligned16(W_UV) || !aligned16(out) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
     const TcWs lay = tc_ws_layout(B, n_q, H);
     if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
@@ -174,21 +174,21 @@ mla_status mla_decode_finish(const int64_t* seq_start, const int32_t* kv_len, in
     if (pg <= 0) return MLA_ERR_CUDA;
     const char* ws = static_cast<const char*>(workspace);
     return cuda_status(launch_combine_tc(reinterpret_cast<const float*>(ws + lay.o_part),
-                                         reinterpret_cast<const float2*>(ws + lay.ml_part), kv_len, seq_start,
-                                         cap_tokens, B, n_q, H, pg, lay.slots, static_cast<const uint16_t*>(W_UV),
+                                         reinterpret_cast<const float2*>(ws + lay.ml_part), kv_len, seq_block,
+                                         cap_blocks, B, n_q, H, pg, lay.slots, static_cast<const uint16_t*>(W_UV),
                                          static_cast<uint16_t*>(out), lse_out, static_cast<cudaStream_t>(stream)));
 }
 
-mla_status mla_decode(const void* q, const void* cache, int64_t cap_tokens, const int64_t* seq_start,
+mla_status mla_decode(const void* q, const void* cache, int64_t cap_blocks, const int64_t* seq_block,
                       const int32_t* kv_len, const void* W_UV, int B, int n_q, int H, float scale, int num_splits,
                       void* workspace, size_t ws_bytes, void* out, float* lse_out, int32_t* dev_status,
                       mla_stream stream) {
     if (B > 0 && (!W_UV || !out)) return MLA_ERR_INVALID_ARG;
     if (B > 0 && (!aligned16(W_UV) || !aligned16(out))) return MLA_ERR_INVALID_ARG;
-    mla_status st = mla_decode_attend(q, cache, cap_tokens, seq_start, kv_len, B, n_q, H, scale, num_splits,
+    mla_status st = mla_decode_attend(q, cache, cap_blocks, seq_block, kv_len, B, n_q, H, scale, num_splits,
                                       workspace, ws_bytes, dev_status, stream);
     if (st != MLA_OK || B == 0) return st;
-    return mla_decode_finish(seq_start, kv_len, cap_tokens, W_UV, B, n_q, H, num_splits, workspace, ws_bytes, out,
+    return mla_decode_finish(seq_block, kv_len, cap_blocks, W_UV, B, n_q, H, num_splits, workspace, ws_bytes, out,
                              lse_out, stream);
 }
 
@@ -198,15 +198,15 @@ size_t mla_decode_cudacore_workspace_bytes(int B, int n_q, int H, int num_splits
     return decode_ws_layout(B, n_q, H, S).total;
 }
 
-mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_tokens, const int64_t* seq_start,
+mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_blocks, const int64_t* seq_block,
                                const int32_t* kv_len, const void* W_UV, int B, int n_q, int H, float scale,
                                int num_splits, void* workspace, size_t ws_bytes, void* out, float* lse_out,
                                int32_t* dev_status, mla_stream stream) {
-    mla_status st = check_decode_shape(B, cap_tokens, n_q, H, num_splits);
+    mla_status st = check_decode_shape(B, cap_blocks, n_q, H, num_splits);
     if (st != MLA_OK) return st;
     if (!(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
     if (B == 0) return MLA_OK;
-    if (!q || !cache || !seq_start || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!q || !cache || !seq_block || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(cache) || !aligned16(W_UV) || !aligned16(out) || !aligned16(workspace))
         return MLA_ERR_INVALID_ARG;
     const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
@@ -215,8 +215,8 @@ mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_tok
     float* o_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.o_part);
     float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.lse_part);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_decode_simt(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(cache),
-                                       cap_tokens, seq_start, kv_len, B, n_q, H, scale, S, o_part, lse_part,
+    cudaError_t e = launch_decode_simt(static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(cache),
+                                       cap_blocks, seq_block, kv_len, B, n_q, H, scale, S, o_part, lse_part,
                                        dev_status, cs);
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     return cuda_status(launch_combine(o_part, lse_part, B * n_q, H, S, static_cast<const uint16_t*>(W_UV), out,

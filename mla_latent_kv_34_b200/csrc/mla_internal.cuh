@@ -15,6 +15,14 @@ constexpr int kDh = 128;           // head width d_h
 constexpr int kRow = kDc + kDr;    // packed cache row (576 bf16 = 1152 B)
 constexpr int kMaxHeads = 128;
 constexpr int kMaxNq = 16;
+constexpr int kBlockTokens = MLA_BLOCK_TOKENS;  // tokens per cache block
+constexpr int kBlockBytes = MLA_BLOCK_BYTES;    // 9 chunks x [64 rows x 128 B]
+static_assert(kBlockBytes == 9 * kBlockTokens * 128, "block layout");
+
+// Byte offset of column c of row r inside a cache block (128-byte swizzle per 64-column chunk).
+__host__ __device__ __forceinline__ int block_offset(int r, int c) {
+    return (c >> 6) * 8192 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2;
+}
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -37,7 +45,7 @@ __device__ __forceinline__ void report(int32_t* dev_status, int32_t bit) {
 }
 
 // Host-side launch wrappers (one per kernel file).
-cudaError_t launch_append_cache(uint16_t* cache, int64_t cap, const int64_t* seq_start, const int32_t* seq_idx,
+cudaError_t launch_append_cache(uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block, const int32_t* seq_idx,
                                 const int32_t* pos, const uint16_t* c_kv, const uint16_t* k_rope,
                                 const float* rope_table, int64_t rope_len, int T, int32_t* dev_status,
                                 cudaStream_t stream);
@@ -46,7 +54,7 @@ cudaError_t launch_absorb_q(const uint16_t* q_nope, const uint16_t* q_rope, cons
                             const uint16_t* W_UK, const float* rope_table, int64_t rope_len, int T, int H,
                             uint16_t* q_out, int32_t* dev_status, cudaStream_t stream);
 
-cudaError_t launch_decode_simt(const uint16_t* q, const uint16_t* cache, int64_t cap, const int64_t* seq_start,
+cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
                                const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,
                                float* o_part, float* lse_part, int32_t* dev_status, cudaStream_t stream);
 
@@ -56,11 +64,11 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int T, in
 // Tensor-core decode (decode_tc.cu) and the merge of its segments (combine.cu).
 int decode_tc_max_clusters();
 int decode_tc_clusters();
-cudaError_t launch_decode_tc(const uint16_t* q, const uint16_t* cache, int64_t cap, const int64_t* seq_start,
+cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
                              const int32_t* kv_len, int B, int n_q, int H, float scale, int clusters_per_group,
                              float* o_part, float2* ml_part, int slots, int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_combine_tc(const float* o_part, const float2* ml_part, const int32_t* kv_len,
-                              const int64_t* seq_start, int64_t cap, int B, int n_q, int H, int P_g, int slots,
+                              const int64_t* seq_block, int64_t cap_blocks, int B, int n_q, int H, int P_g, int slots,
                               const uint16_t* W_UV, uint16_t* out, float* lse_out, cudaStream_t stream);
 
 }  // namespace mla

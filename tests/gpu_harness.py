@@ -13,6 +13,32 @@ import mla_latent_kv_34_b200 as mla
 from oracle import naive as on
 
 NAN_BF16 = 0x7FC0  # quiet NaN pattern put in cache rows no sequence owns
+BLOCK_TOKENS, BLOCK_BYTES = 64, 73728
+
+
+def _block_index_map() -> np.ndarray:
+    """[64, 576] uint16 offsets inside a cache block of (row r, column c), per the mla.h layout."""
+    r = np.arange(64)[:, None]
+    c = np.arange(576)[None, :]
+    byte = (c // 64) * 8192 + r * 128 + ((((c % 64) // 8) ^ (r % 8)) * 16) + (c % 8) * 2
+    return (byte // 2).astype(np.int64)
+
+
+BLOCK_MAP = _block_index_map()
+
+
+def unpack_rows(cache_u16: np.ndarray, blocks: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """Logical [n, 576] rows (bf16 bits) of a blocked cache given as uint16 [cap_blocks, 36864]."""
+    return cache_u16[np.asarray(blocks)[:, None], BLOCK_MAP[np.asarray(rows)]]
+
+
+def pack_rows(cache_u16: np.ndarray, blocks: np.ndarray, rows: np.ndarray, values: np.ndarray) -> None:
+    """Inverse of unpack_rows (in place)."""
+    cache_u16[np.asarray(blocks)[:, None], BLOCK_MAP[np.asarray(rows)]] = values
+
+
+def cache_u16(cache: torch.Tensor) -> np.ndarray:
+    return cache.cpu().numpy().view(np.uint16).reshape(cache.shape[0], BLOCK_BYTES // 2)
 
 
 def to_dev_bf16(bits: np.ndarray, dev) -> torch.Tensor:
@@ -32,9 +58,9 @@ def rel_l2(got: np.ndarray, ref: np.ndarray) -> float:
 class Problem:
     cfg: mi.MLAConfig
     lengths: np.ndarray
-    starts: np.ndarray
+    starts: np.ndarray  # first block of each sequence
     cache: torch.Tensor
-    seq_start: torch.Tensor
+    seq_block: torch.Tensor
     kv_len: torch.Tensor
     q_nope: torch.Tensor
     q_rope: torch.Tensor
@@ -54,7 +80,7 @@ class Problem:
     def decode(self, q, num_splits=0, lse=True, path="tc"):
         lse_out = torch.empty((self.T, self.cfg.H), dtype=torch.float32, device=q.device) if lse else None
         fn = mla.decode if path == "tc" else mla.decode_cudacore
-        out = fn(q, self.cache, self.seq_start, self.kv_len, self.W_UV, self.cfg.n_q, self.cfg.scale,
+        out = fn(q, self.cache, self.seq_block, self.kv_len, self.W_UV, self.cfg.n_q, self.cfg.scale,
                  num_splits=num_splits, lse_out=lse_out, dev_status=self.status)
         return out, lse_out
 
@@ -68,36 +94,39 @@ class Problem:
                                self.cfg.n_q, scale=self.cfg.scale, base=self.cfg.rope_base, heads=heads)
 
 
-def build_problem(cfg: mi.MLAConfig, lengths=None, slack_rows: int = 64, dev="cuda",
-                  chunk_rows: int = 1 << 16, gap_rows: int = 0) -> Problem:
-    """Fill a packed cache with every sequence's tokens via mla_append_cache.
+def build_problem(cfg: mi.MLAConfig, lengths=None, slack_blocks: int = 2, dev="cuda",
+                  chunk_rows: int = 1 << 16, gap_blocks: int = 0) -> Problem:
+    """Fill a blocked cache with every sequence's tokens via mla_append_cache.
 
-    Sequences sit back to back from row 0 (or ``gap_rows`` apart); the gaps and
-    ``slack_rows`` extra rows at the end hold NaN so that a kernel reading past
-    a sequence would be noticed.
+    Sequences occupy consecutive blocks from block 0 (``gap_blocks`` apart);
+    every byte not written by an append (the tails of last blocks, the gaps and
+    ``slack_blocks`` extra blocks) holds the bf16 NaN pattern, so a kernel that
+    used a row outside a sequence would be noticed.
     """
     lengths = mi.kv_lengths(cfg) if lengths is None else np.asarray(lengths, dtype=np.int64)
     pool_starts = mi.seq_starts(lengths)            # rows in the generator's packed pool
-    starts = pool_starts + gap_rows * np.arange(cfg.B, dtype=np.int64)
+    nblk = (lengths + BLOCK_TOKENS - 1) // BLOCK_TOKENS
+    seq_block = np.zeros(cfg.B, dtype=np.int64)
+    if cfg.B > 1:
+        seq_block[1:] = np.cumsum(nblk[:-1] + gap_blocks)
+    cap_blocks = int(seq_block[-1] + nblk[-1]) + slack_blocks
     N = int(lengths.sum())
-    cap = N + gap_rows * cfg.B + slack_rows
-    cache = torch.full((cap, mi.D_ROW), NAN_BF16, dtype=torch.int16, device=dev)
-    cache = cache.view(torch.bfloat16)
+    cache = torch.full((cap_blocks, BLOCK_BYTES // 2), NAN_BF16, dtype=torch.int16, device=dev).view(torch.uint8)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     rope_tab = mla.rope_table(int(lengths.max()), cfg.rope_base, dev)
-    seq_start = torch.from_numpy(starts).to(dev)
+    seq_block_t = torch.from_numpy(seq_block).to(dev)
     # per-row (sequence, position) of the whole pool
     seq_of_row = np.repeat(np.arange(cfg.B, dtype=np.int32), lengths)
     pos_of_row = (np.arange(N, dtype=np.int64) - np.repeat(pool_starts, lengths)).astype(np.int32)
     for r0 in range(0, N, chunk_rows):
         n = min(chunk_rows, N - r0)
         c, k = mi.token_rows(cfg, r0, n)
-        mla.append_cache(cache, seq_start, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
+        mla.append_cache(cache, seq_block_t, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
                          torch.from_numpy(pos_of_row[r0:r0 + n]).to(dev), to_dev_bf16(c, dev),
                          to_dev_bf16(k, dev), rope_tab, status)
     qn, qr = mi.queries(cfg)
     q_pos = np.concatenate([lengths[b] - cfg.n_q + np.arange(cfg.n_q) for b in range(cfg.B)]).astype(np.int32)
-    return Problem(cfg, lengths, starts, cache, seq_start,
+    return Problem(cfg, lengths, seq_block, cache, seq_block_t,
                    torch.from_numpy(lengths.astype(np.int32)).to(dev),
                    to_dev_bf16(qn, dev), to_dev_bf16(qr, dev), torch.from_numpy(q_pos).to(dev),
                    to_dev_bf16(mi.weights(cfg, "uk"), dev), to_dev_bf16(mi.weights(cfg, "uv"), dev),

@@ -50,12 +50,13 @@ def _check_decode(prob, out, lse, seqs, heads=None, label=""):
 # ----------------------------------------------------------------- append
 
 def test_append_bit_exact_with_canary(cuda_ok, H):
+    """Appended rows equal the fp32 emulation bit for bit; no other byte changes."""
     dev = "cuda"
     import mla_latent_kv_34_b200 as mla
-    cap = 5000
-    canary = np.full((cap, 576), 0xA5A5, dtype=np.uint16)
-    cache = H.to_dev_bf16(canary, dev)
-    starts = np.array([0, 1000, 2500, 4000], dtype=np.int64)
+    cap_blocks = 80
+    canary = np.full((cap_blocks, H.BLOCK_BYTES // 2), 0xA5A5, dtype=np.uint16)
+    cache = torch.from_numpy(canary.view(np.int16).copy()).to(dev).view(torch.uint8)
+    seq_block = np.array([0, 17, 40, 63], dtype=np.int64)
     rng = np.random.default_rng(1)
     T = 777
     seq_idx = rng.integers(0, 4, T).astype(np.int32)
@@ -63,17 +64,23 @@ def test_append_bit_exact_with_canary(cuda_ok, H):
     pos = np.empty(T, dtype=np.int32)
     for s in range(4):
         idx = np.where(seq_idx == s)[0]
-        pos[idx] = rng.choice(900, len(idx), replace=False)
+        pos[idx] = rng.choice(1000, len(idx), replace=False)
     c = mi.normal_bf16(77, 1, 0, T * 512).reshape(T, 512)
     k = mi.normal_bf16(77, 2, 0, T * 64).reshape(T, 64)
     tab = mla.rope_table(1000, 10000.0, dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    mla.append_cache(cache, torch.from_numpy(starts).to(dev), torch.from_numpy(seq_idx).to(dev),
+    mla.append_cache(cache, torch.from_numpy(seq_block).to(dev), torch.from_numpy(seq_idx).to(dev),
                      torch.from_numpy(pos).to(dev), H.to_dev_bf16(c, dev), H.to_dev_bf16(k, dev), tab, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    ref = oapp.append_rows(canary, starts, seq_idx, pos, c, k)
-    np.testing.assert_array_equal(_bits(cache), ref)
+    # logical rows from the oracle's fp32 emulation, placed per the documented block layout
+    rows = np.concatenate([c, oapp.rotate_k_bits(k, pos)], axis=1)
+    expect = canary.copy()
+    blk = seq_block[seq_idx] + pos // 64
+    H.pack_rows(expect, blk, pos % 64, rows)
+    got = H.cache_u16(cache)
+    np.testing.assert_array_equal(H.unpack_rows(got, blk, pos % 64), rows)
+    np.testing.assert_array_equal(got, expect)
 
 
 def test_append_large_positions_bit_exact(cuda_ok, H):
@@ -81,15 +88,15 @@ def test_append_large_positions_bit_exact(cuda_ok, H):
     dev = "cuda"
     T = 512
     pos = (131071 - 255 * (T - 1 - np.arange(T, dtype=np.int64))).astype(np.int32)
-    cap = int(pos.max()) + 1
-    cache = torch.zeros((cap, 576), dtype=torch.bfloat16, device=dev)
+    cap_blocks = int(pos.max()) // 64 + 1
+    cache = mla.new_cache(cap_blocks, dev)
     c = mi.normal_bf16(78, 1, 0, T * 512).reshape(T, 512)
     k = mi.normal_bf16(78, 2, 0, T * 64).reshape(T, 64)
     tab = mla.rope_table(131072, 10000.0, dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     mla.append_cache(cache, torch.zeros(1, dtype=torch.int64, device=dev), torch.zeros(T, dtype=torch.int32, device=dev),
                      torch.from_numpy(pos).to(dev), H.to_dev_bf16(c, dev), H.to_dev_bf16(k, dev), tab, st)
-    got = _bits(cache[torch.from_numpy(pos.astype(np.int64)).to(dev)])
+    got = H.unpack_rows(H.cache_u16(cache), pos // 64, pos % 64)
     np.testing.assert_array_equal(got[:, :512], c)
     np.testing.assert_array_equal(got[:, 512:], oapp.rotate_k_bits(k, pos))
     assert int(st.item()) == 0
@@ -98,16 +105,19 @@ def test_append_large_positions_bit_exact(cuda_ok, H):
 def test_append_out_of_range_is_reported_and_skipped(cuda_ok, H):
     import mla_latent_kv_34_b200 as mla
     dev = "cuda"
-    cache = torch.zeros((10, 576), dtype=torch.bfloat16, device=dev)
-    tab = mla.rope_table(64, 10000.0, dev)
+    cache = torch.zeros((3, H.BLOCK_BYTES), dtype=torch.uint8, device=dev)
+    tab = mla.rope_table(256, 10000.0, dev)
     c = torch.ones((2, 512), dtype=torch.bfloat16, device=dev)
     k = torch.ones((2, 64), dtype=torch.bfloat16, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    mla.append_cache(cache, torch.tensor([0, 8], device=dev), torch.tensor([0, 1], dtype=torch.int32, device=dev),
-                     torch.tensor([3, 5], dtype=torch.int32, device=dev), c, k, tab, st)
+    # sequence 1 starts at block 2: position 70 lands in block 3 = out of range
+    mla.append_cache(cache, torch.tensor([0, 2], device=dev), torch.tensor([0, 1], dtype=torch.int32, device=dev),
+                     torch.tensor([3, 70], dtype=torch.int32, device=dev), c, k, tab, st)
     torch.cuda.synchronize()
     assert int(st.item()) & 0x1
-    assert cache[3].float().sum().item() != 0 and cache[9].float().abs().sum().item() == 0
+    u = H.cache_u16(cache)
+    assert np.any(H.unpack_rows(u, [0], [3]) != 0)
+    assert np.all(u[1:] == 0)
     st.zero_()
     mla.append_cache(cache, torch.tensor([0], device=dev), torch.tensor([0], dtype=torch.int32, device=dev),
                      torch.tensor([9], dtype=torch.int32, device=dev), c[:1], k[:1], tab[:5], st)
@@ -194,7 +204,7 @@ def test_decode_split_invariance(cuda_ok, H, splits):
 def test_decode_ignores_rows_outside_sequences(cuda_ok, H):
     """NaN rows between and after sequences never leak into any result."""
     cfg = mi.MLAConfig("gaps", B=5, H=128, n_q=2, L=None, L_max=400, seed=66)
-    prob = H.build_problem(cfg, gap_rows=37)
+    prob = H.build_problem(cfg, gap_blocks=3)
     out, lse = prob.decode(prob.absorb())
     torch.cuda.synchronize()
     assert int(prob.status.item()) == 0
