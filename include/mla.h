@@ -99,7 +99,8 @@ mla_status mla_rope_table_fill(float* table_host, int64_t rope_len, double base)
  *                                already rotated and is copied)
  *   W_UK    bf16 [H, 128, 512]   per-head up-projection (k^C = W^UK_h c)
  *   q_out   bf16 [T, H, 576]     [ (W^UK_h)^T q_nope (512) | R_pos q^R (64) ]
- * fp32 accumulation, one rounding to bf16 per output element.
+ * fp32 accumulation (tensor cores), one rounding to bf16 per output element;
+ * the q^R rotation uses the same fp32 arithmetic as mla_append_cache.
  */
 mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* pos,
                         const void* W_UK, const float* rope_table, int64_t rope_len,
@@ -183,7 +184,7 @@ mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_block
 mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, int64_t cap_blocks,
                              const void* W_UV, int B, int n_q, int H, int num_splits,
                              void* workspace, size_t ws_bytes, void* out, float* lse_out,
-                             mla_stream stream);
+                             int32_t* dev_status, mla_stream stream);
 
 /*
  * mla_decode_cudacore -- the same decode step computed on CUDA cores (fp32

@@ -38,7 +38,7 @@ _SIGS = {
     "mla_decode_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
     "mla_decode": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
     "mla_decode_attend": ([_p, _p, _i64, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p], _i32),
-    "mla_decode_finish": ([_p, _p, _i64, _p, _i32, _i32, _i32, _i32, _p, _sz, _p, _p, _p], _i32),
+    "mla_decode_finish": ([_p, _p, _i64, _p, _i32, _i32, _i32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
     "mla_decode_cudacore_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
     "mla_decode_cudacore": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p],
                             _i32),
@@ -169,7 +169,7 @@ def decode_attend(q, cache, seq_block, kv_len, n_q: int, scale: float, num_split
 
 
 def decode_finish(seq_block, kv_len, cache, W_UV, n_q: int, num_splits: int, workspace, out, lse_out=None,
-                  stream=None):
+                  dev_status=None, stream=None):
     """Phase 2 of decode: merge the partials, apply W^UV into ``out`` bf16 [B*n_q, H, 128]."""
     B = kv_len.shape[0]
     H = W_UV.shape[0]
@@ -178,7 +178,7 @@ def decode_finish(seq_block, kv_len, cache, W_UV, n_q: int, num_splits: int, wor
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(out, torch.bfloat16, (B * n_q, H, D_H), "out"), _ptr(lse_out, torch.float32, (B * n_q, H), "lse_out"),
-        _stream(stream)))
+        _ptr(dev_status, torch.int32, None, "dev_status"), _stream(stream)))
     return out
 
 

@@ -99,124 +99,4 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int T, in
 }
 
 
-// ---------------------------------------------------------------------------
-// Merge of the tensor-core decode's segments.  Each segment s of a sequence
-// holds its unnormalised latent sum O_s (relative to its running max m_s,
-// log2 units) and its softmax denominator l_s; with M = max_s m_s:
-//   o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,
-//   lse = ln 2 * (M + log2 sum_s 2^(m_s - M) l_s).
-// The segments of sequence b are the pieces of the equal cluster ranges
-// [p Nt / P, (p+1) Nt / P) of the global tile space that overlap its tiles.
-
-__device__ __forceinline__ int tc_seq_tiles(const int32_t* kv_len, const int64_t* seq_block, int64_t cap_blocks,
-                                            int n_q, int b) {
-    const int L = kv_len[b];
-    if (L < n_q) return 0;
-    const int64_t s = seq_block[b];
-    const int nt = (L + kBlockTokens - 1) / kBlockTokens;
-    if (s < 0 || s + nt > cap_blocks) return 0;
-    return nt;
-}
-
-__global__ void __launch_bounds__(256) combine_tc_kernel(
-    const float* __restrict__ o_part, const float2* __restrict__ ml_part, const int32_t* __restrict__ kv_len,
-    const int64_t* __restrict__ seq_block, int64_t cap_blocks, int B, int n_q, int H, int P_g, int slots,
-    const uint16_t* __restrict__ W_UV, uint16_t* __restrict__ out, float* __restrict__ lse_out) {
-    __shared__ float ol[kCombTok][kDc];
-    __shared__ int red[2][8];
-    __shared__ int ts_of[kCombTok + 1], nt_of[kCombTok + 1];
-    const int h = blockIdx.x;
-    const int T = B * n_q;
-    const int t0 = blockIdx.y * kCombTok;
-    const int nt = min(kCombTok, T - t0);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b_lo = t0 / n_q;
-    const int b_hi = (t0 + nt - 1) / n_q;
-    // total tiles and tiles before b_lo
-    int s_all = 0, s_before = 0;
-    for (int b = tid; b < B; b += blockDim.x) {
-        const int v = tc_seq_tiles(kv_len, seq_block, cap_blocks, n_q, b);
-        s_all += v;
-        s_before += (b < b_lo) ? v : 0;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        s_all += __shfl_xor_sync(0xffffffffu, s_all, o);
-        s_before += __shfl_xor_sync(0xffffffffu, s_before, o);
-    }
-    if (lane == 0) {
-        red[0][warp] = s_all;
-        red[1][warp] = s_before;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int a = 0, bb = 0;
-        for (int w = 0; w < 8; ++w) {
-            a += red[0][w];
-            bb += red[1][w];
-        }
-        red[0][0] = a;
-        int ts = bb;
-        for (int b = b_lo; b <= b_hi; ++b) {
-            const int v = tc_seq_tiles(kv_len, seq_block, cap_blocks, n_q, b);
-            ts_of[b - b_lo] = ts;
-            nt_of[b - b_lo] = v;
-            ts += v;
-        }
-    }
-    __syncthreads();
-    const int Nt = red[0][0];
-    for (int t = 0; t < nt; ++t) {
-        const int tt = t0 + t;
-        const int b = tt / n_q, j = tt % n_q;
-        const int rr = j * H + h;
-        const int g = rr / 128, r = rr % 128;
-        const int ts = ts_of[b - b_lo], ntb = nt_of[b - b_lo];
-        float o0 = 0.f, o1 = 0.f, z = 0.f, M = -CUDART_INF_F;
-        if (ntb > 0 && Nt > 0) {
-            const int p_first = static_cast<int>((static_cast<int64_t>(ts + 1) * P_g - 1) / Nt);
-            const int p_last = static_cast<int>((static_cast<int64_t>(ts + ntb) * P_g - 1) / Nt);
-            const int64_t gbase = static_cast<int64_t>(g) * slots;
-            for (int pass = 0; pass < 2; ++pass) {
-                for (int p = p_first; p <= p_last; ++p) {
-                    const int lo = static_cast<int>((static_cast<int64_t>(p) * Nt) / P_g);
-                    const int hi = static_cast<int>((static_cast<int64_t>(p + 1) * Nt) / P_g);
-                    if (max(lo, ts) >= min(hi, ts + ntb)) continue;
-                    const int64_t row = (gbase + b + p) * 128 + r;
-                    const float2 ml = ml_part[row];
-                    if (pass == 0) {
-                        M = fmaxf(M, ml.x);
-                        continue;
-                    }
-                    if (ml.x == -CUDART_INF_F) continue;
-                    const float w = exp2f(ml.x - M);
-                    const float2 v = *reinterpret_cast<const float2*>(o_part + row * kDc + 2 * tid);
-                    o0 = fmaf(w, v.x, o0);
-                    o1 = fmaf(w, v.y, o1);
-                    z = fmaf(w, ml.y, z);
-                }
-                if (M == -CUDART_INF_F) break;
-            }
-        }
-        const float inv = (z > 0.f) ? 1.f / z : 0.f;
-        ol[t][2 * tid] = o0 * inv;
-        ol[t][2 * tid + 1] = o1 * inv;
-        if (tid == 0 && lse_out)
-            lse_out[static_cast<int64_t>(tt) * H + h] = (z > 0.f) ? (M + log2f(z)) * 0.69314718055994530942f
-                                                                  : -CUDART_INF_F;
-    }
-    __syncthreads();
-    up_project_block(ol, nt, t0, h, H, W_UV, out);
-}
-
-cudaError_t launch_combine_tc(const float* o_part, const float2* ml_part, const int32_t* kv_len,
-                              const int64_t* seq_block, int64_t cap_blocks, int B, int n_q, int H, int P_g, int slots,
-                              const uint16_t* W_UV, uint16_t* out, float* lse_out, cudaStream_t stream) {
-    const int T = B * n_q;
-    dim3 grid(H, (T + kCombTok - 1) / kCombTok);
-    combine_tc_kernel<<<grid, 256, 0, stream>>>(o_part, ml_part, kv_len, seq_block, cap_blocks, B, n_q, H, P_g, slots, W_UV,
-                                                out, lse_out);
-    return cudaGetLastError();
-}
-
 }  // namespace mla

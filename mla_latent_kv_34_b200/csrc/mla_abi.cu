@@ -115,7 +115,7 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* p
     if (T == 0) return MLA_OK;
     if (!q_nope || !q_rope || !W_UK || !q_out || (pos && !rope_table)) return MLA_ERR_INVALID_ARG;
     if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(W_UK) || !aligned16(q_out)) return MLA_ERR_INVALID_ARG;
-    return cuda_status(launch_absorb_q(static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_rope),
+    return cuda_status(launch_absorb_tc(static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_rope),
                                        pos, static_cast<const uint16_t*>(W_UK), rope_table, rope_len, T, H,
                                        static_cast<uint16_t*>(q_out), dev_status,
                                        static_cast<cudaStream_t>(stream)));
@@ -162,7 +162,7 @@ mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_block
 
 mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, int64_t cap_blocks, const void* W_UV,
                              int B, int n_q, int H, int num_splits, void* workspace, size_t ws_bytes, void* out,
-                             float* lse_out, mla_stream stream) {
+                             float* lse_out, int32_t* dev_status, mla_stream stream) {
     mla_status st = check_decode_shape(B, cap_blocks, n_q, H, num_splits);
     if (st != MLA_OK) return st;
     if (B == 0) return MLA_OK;
@@ -173,10 +173,11 @@ mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, in
     const int pg = tc_clusters_per_group(lay.G, num_splits);
     if (pg <= 0) return MLA_ERR_CUDA;
     const char* ws = static_cast<const char*>(workspace);
-    return cuda_status(launch_combine_tc(reinterpret_cast<const float*>(ws + lay.o_part),
-                                         reinterpret_cast<const float2*>(ws + lay.ml_part), kv_len, seq_block,
-                                         cap_blocks, B, n_q, H, pg, lay.slots, static_cast<const uint16_t*>(W_UV),
-                                         static_cast<uint16_t*>(out), lse_out, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_finish_tc(reinterpret_cast<const float*>(ws + lay.o_part),
+                                        reinterpret_cast<const float2*>(ws + lay.ml_part), kv_len, seq_block,
+                                        cap_blocks, B, n_q, H, pg, lay.slots, static_cast<const uint16_t*>(W_UV),
+                                        static_cast<uint16_t*>(out), lse_out, dev_status,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 mla_status mla_decode(const void* q, const void* cache, int64_t cap_blocks, const int64_t* seq_block,
@@ -189,7 +190,7 @@ mla_status mla_decode(const void* q, const void* cache, int64_t cap_blocks, cons
                                       workspace, ws_bytes, dev_status, stream);
     if (st != MLA_OK || B == 0) return st;
     return mla_decode_finish(seq_block, kv_len, cap_blocks, W_UV, B, n_q, H, num_splits, workspace, ws_bytes, out,
-                             lse_out, stream);
+                             lse_out, dev_status, stream);
 }
 
 size_t mla_decode_cudacore_workspace_bytes(int B, int n_q, int H, int num_splits) {

@@ -50,9 +50,9 @@ cudaError_t launch_append_cache(uint8_t* cache, int64_t cap_blocks, const int64_
                                 const float* rope_table, int64_t rope_len, int T, int32_t* dev_status,
                                 cudaStream_t stream);
 
-cudaError_t launch_absorb_q(const uint16_t* q_nope, const uint16_t* q_rope, const int32_t* pos,
-                            const uint16_t* W_UK, const float* rope_table, int64_t rope_len, int T, int H,
-                            uint16_t* q_out, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_absorb_tc(const uint16_t* q_nope, const uint16_t* q_rope, const int32_t* pos, const uint16_t* W_UK,
+                             const float* rope_table, int64_t rope_len, int T, int H, uint16_t* q_out,
+                             int32_t* dev_status, cudaStream_t stream);
 
 cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
                                const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,
@@ -61,14 +61,14 @@ cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int T, int H, int splits,
                            const uint16_t* W_UV, void* out, float* lse_out, cudaStream_t stream);
 
-// Tensor-core decode (decode_tc.cu) and the merge of its segments (combine.cu).
+// Tensor-core decode (decode_tc.cu); projections and the merge of its segments (proj_tc.cu).
 int decode_tc_max_clusters();
 int decode_tc_clusters();
 cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
                              const int32_t* kv_len, int B, int n_q, int H, float scale, int clusters_per_group,
                              float* o_part, float2* ml_part, int slots, int32_t* dev_status, cudaStream_t stream);
-cudaError_t launch_combine_tc(const float* o_part, const float2* ml_part, const int32_t* kv_len,
-                              const int64_t* seq_block, int64_t cap_blocks, int B, int n_q, int H, int P_g, int slots,
-                              const uint16_t* W_UV, uint16_t* out, float* lse_out, cudaStream_t stream);
+cudaError_t launch_finish_tc(const float* o_part, const float2* ml_part, const int32_t* kv_len, const int64_t* seq_block,
+                             int64_t cap_blocks, int B, int n_q, int H, int P_g, int slots, const uint16_t* W_UV,
+                             uint16_t* out, float* lse_out, int32_t* dev_status, cudaStream_t stream);
 
 }  // namespace mla
