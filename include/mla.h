@@ -187,6 +187,32 @@ mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, in
                              int32_t* dev_status, mla_stream stream);
 
 /*
+ * mla_decode_static -- mla_decode without a workspace argument: the step's
+ * segment partials go to one scratch buffer owned by the library (a static
+ * device array of MLA_DECODE_STATIC_SCRATCH_BYTES per device).  Neither
+ * paper has a counterpart; this is a convenience of the library for callers
+ * that cannot allocate device memory where they decode (a frozen memory
+ * pool, a thread that must not enter the CUDA allocator, code without any
+ * allocator).  Nothing on this path allocates.
+ *   Arguments, layouts and results are those of mla_decode.
+ *   Limit: shapes with mla_decode_workspace_bytes(B, n_q, H, num_splits) >
+ *   MLA_DECODE_STATIC_SCRATCH_BYTES return MLA_ERR_WORKSPACE and launch
+ *   nothing (with 74 CTA pairs and 128 query rows per group this allows
+ *   groups * (B + 74) <= 127, e.g. B <= 53 at H = 128, n_q = 1).
+ *   Set-up: the first call on a device looks the buffer up (and may load the
+ *   library's device code there); make it before any stream capture.
+ *   Zeroing: none needed; every partial read is written in the same call.
+ *   Races: one buffer per device, so calls that can overlap on a device
+ *   (other streams, unordered host threads) corrupt each other's partials;
+ *   calls ordered on one stream are safe.
+ */
+#define MLA_DECODE_STATIC_SCRATCH_BYTES (32u << 20)
+mla_status mla_decode_static(const void* q, const void* cache, int64_t cap_blocks,
+                             const int64_t* seq_block, const int32_t* kv_len, const void* W_UV,
+                             int B, int n_q, int H, float scale, int num_splits,
+                             void* out, float* lse_out, int32_t* dev_status, mla_stream stream);
+
+/*
  * mla_decode_cudacore -- the same decode step computed on CUDA cores (fp32
  * FMA, split-KV over `num_splits` equal key ranges per sequence, 0 =
  * automatic) instead of the tensor cores.  Same arguments and results as

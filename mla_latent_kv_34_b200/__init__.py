@@ -39,6 +39,7 @@ _SIGS = {
     "mla_decode": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
     "mla_decode_attend": ([_p, _p, _i64, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p], _i32),
     "mla_decode_finish": ([_p, _p, _i64, _p, _i32, _i32, _i32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
+    "mla_decode_static": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _p, _p, _p], _i32),
     "mla_decode_cudacore_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
     "mla_decode_cudacore": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p],
                             _i32),
@@ -150,6 +151,31 @@ def decode(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits
         _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, float(scale), num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _ptr(out, torch.bfloat16, (T, H, D_H), "out"), _ptr(lse_out, torch.float32, (T, H), "lse_out"),
+        _ptr(dev_status, torch.int32, None, "dev_status"), _stream(stream)))
+    return out
+
+
+DECODE_STATIC_SCRATCH_BYTES = 32 << 20  # MLA_DECODE_STATIC_SCRATCH_BYTES
+
+
+def decode_static(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
+                  out=None, lse_out=None, dev_status=None, stream=None):
+    """``decode`` with the library's own scratch (no workspace; ``out`` must be given to avoid any allocation).
+
+    Calls that can overlap on one device race on that scratch; the first call per device must precede any
+    stream capture.
+    """
+    B = kv_len.shape[0]
+    T, H = q.shape[0], q.shape[1]
+    if T != B * n_q:
+        raise MLAError("q rows must equal len(kv_len) * n_q")
+    if out is None:
+        out = torch.empty((T, H, D_H), dtype=torch.bfloat16, device=q.device)
+    _check(lib.mla_decode_static(
+        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0],
+        _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, float(scale), num_splits,
         _ptr(out, torch.bfloat16, (T, H, D_H), "out"), _ptr(lse_out, torch.float32, (T, H), "lse_out"),
         _ptr(dev_status, torch.int32, None, "dev_status"), _stream(stream)))
     return out
