@@ -19,15 +19,16 @@
  * sequence (1..16), T = B * n_q query rows (row t = b * n_q + j).
  *
  * Latent cache layout (blocked).  The cache is an array of blocks of
- * MLA_BLOCK_TOKENS = 64 tokens, MLA_BLOCK_BYTES = 73728 bytes each.  Token
- * `pos` of sequence b lives in block seq_block[b] + pos / 64, at row
- * r = pos % 64; its 576 bf16 values [c^KV (0..511) | rotated k^R (512..575)]
+ * MLA_BLOCK_TOKENS = 128 tokens, MLA_BLOCK_BYTES = 147456 bytes each.  Token
+ * `pos` of sequence b lives in block seq_block[b] + pos / 128, at row
+ * r = pos % 128; its 576 bf16 values [c^KV (0..511) | rotated k^R (512..575)]
  * are stored as nine 64-column chunks, column c at byte offset
- *     (c / 64) * 8192 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2
- * within the block: each chunk is a [64 rows x 128 bytes] tile whose 16-byte
- * units are permuted by the row index (the 128-byte swizzle), so that one
- * contiguous copy places a block in shared memory exactly as the tensor-core
- * operands are read.  Each sequence occupies ceil(L_b / 64) consecutive blocks.
+ *     (c / 64) * 16384 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2
+ * within the block: each chunk is a [128 rows x 128 bytes] tile whose 16-byte
+ * units are permuted by the row index (the 128-byte swizzle), so that
+ * contiguous copies place a block in shared memory exactly as the tensor-core
+ * operands are read (128 tokens per block make the score MMA 128 wide).  Each
+ * sequence occupies ceil(L_b / 128) consecutive blocks.
  *
  * Conventions for every entry point:
  *   - All tensor arguments are DEVICE pointers to caller-owned memory, dense
@@ -60,8 +61,8 @@ extern "C" {
 
 typedef void* mla_stream; /* cudaStream_t */
 
-#define MLA_BLOCK_TOKENS 64
-#define MLA_BLOCK_BYTES 73728
+#define MLA_BLOCK_TOKENS 128
+#define MLA_BLOCK_BYTES 147456
 
 typedef enum {
     MLA_OK = 0,
@@ -111,7 +112,7 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* p
  * ("两张账" page: only c^KV and k^R are cached; explainer 2.2.2: k^R is
  *  cached already rotated.)
  *   cache      cap_blocks blocks of MLA_BLOCK_BYTES (layout above); token i
- *              goes to block seq_block[seq_idx[i]] + pos[i] / 64, row pos[i] % 64
+ *              goes to block seq_block[seq_idx[i]] + pos[i] / 128, row pos[i] % 128
  *   seq_block  int64 [*]  first cache block of each sequence
  *   seq_idx    int32 [T]  sequence of token i
  *   pos        int32 [T]  position of token i within its sequence
@@ -145,13 +146,13 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
  *  content/position inner product.)
  *   q          bf16 [B*n_q, H, 576]   from mla_absorb_q
  *   cache      cap_blocks blocks (layout above); sequence b occupies blocks
- *              seq_block[b] .. seq_block[b] + ceil(kv_len[b] / 64) - 1 (kv_len
+ *              seq_block[b] .. seq_block[b] + ceil(kv_len[b] / 128) - 1 (kv_len
  *              counts the n_q tokens of this step, already appended)
  *   seq_block  int64 [B];  kv_len int32 [B]
  *   W_UV       bf16 [H, 128, 512]
  *   scale      softmax scale, 1/sqrt(d_h + d_h^R) = 1/sqrt(192) for V2 shapes
  *   num_splits 0: use every SM.  n > 0: at most n CTA pairs per group of 128
- *              query rows.  The (sequence, 64-token tile) space is cut into
+ *              query rows.  The (sequence, 128-token tile) space is cut into
  *              equal contiguous ranges, one per CTA pair; the pieces of a
  *              sequence are merged by log-sum-exp.  Results do not depend on
  *              n beyond fp32 summation order.

@@ -17,8 +17,8 @@ import torch
 
 D_C, D_R, D_H = 512, 64, 128
 D_ROW = D_C + D_R
-BLOCK_TOKENS = 64       # tokens per cache block
-BLOCK_BYTES = 73728     # 9 chunks x [64 rows x 128 bytes]
+BLOCK_TOKENS = 128      # tokens per cache block
+BLOCK_BYTES = 147456    # 9 chunks x [128 rows x 128 bytes]
 
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_b200.so")
 if not os.path.exists(_LIB_PATH):
@@ -120,7 +120,7 @@ def _cache_ptr(cache):
 
 
 def append_cache(cache, seq_block, seq_idx, pos, c_kv, k_rope, rope_tab, dev_status=None, stream=None):
-    """Write c_kv [T,512] and R_pos k_rope [T,64] at token pos of sequence seq_idx (block seq_block[seq_idx] + pos/64)."""
+    """Write c_kv [T,512] and R_pos k_rope [T,64] at token pos of sequence seq_idx (block seq_block[seq_idx] + pos/128)."""
     T = c_kv.shape[0]
     _check(lib.mla_append_cache(
         _cache_ptr(cache), cache.shape[0], _ptr(seq_block, torch.int64, None, "seq_block"),

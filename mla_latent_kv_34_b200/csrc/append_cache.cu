@@ -7,8 +7,8 @@
 // (__fmul_rn / __fadd_rn / __fsub_rn are never contracted into an FMA), then
 // round-to-nearest-even to bf16, so the stored bits are reproducible.
 //
-// Block layout (see mla.h): row r of a 64-token block keeps column c at byte
-// (c / 64) * 8192 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2.
+// Block layout (see mla.h): row r of a 128-token block keeps column c at byte
+// (c / 64) * 16384 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2.
 #include "mla_internal.cuh"
 
 namespace mla {
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(256) append_cache_kernel(
     for (int k = 0; k < 2; ++k) {
         const int w = lane + 32 * k;  // unit index in the row, 0..63
         const int chunk = w >> 3, u = w & 7;
-        *reinterpret_cast<uint4*>(dst + chunk * 8192 + ((u ^ (r & 7)) << 4)) = src4[w];
+        *reinterpret_cast<uint4*>(dst + chunk * kBlockChunk + ((u ^ (r & 7)) << 4)) = src4[w];
     }
     // RoPE pair `lane`: dims (2 lane, 2 lane + 1) -> columns 512 + 2 lane (chunk 8)
     const uint32_t xr = reinterpret_cast<const uint32_t*>(k_rope + static_cast<int64_t>(warp) * kDr)[lane];
@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(256) append_cache_kernel(
     const float y0 = __fsub_rn(__fmul_rn(x0, cs.x), __fmul_rn(x1, cs.y));
     const float y1 = __fadd_rn(__fmul_rn(x0, cs.y), __fmul_rn(x1, cs.x));
     const int u = lane >> 2;  // 16-byte unit within chunk 8
-    *reinterpret_cast<uint32_t*>(dst + 8 * 8192 + ((u ^ (r & 7)) << 4) + (lane & 3) * 4) = pack_bf16x2(y0, y1);
+    *reinterpret_cast<uint32_t*>(dst + 8 * kBlockChunk + ((u ^ (r & 7)) << 4) + (lane & 3) * 4) = pack_bf16x2(y0, y1);
 }
 
 cudaError_t launch_append_cache(uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block, const int32_t* seq_idx,

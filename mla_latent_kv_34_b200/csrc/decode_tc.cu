@@ -7,18 +7,22 @@
 // scores and aggregation both run against the one shared latent cache.
 //
 // Work split.  A cluster of two CTAs (one SM each) owns 128 query rows:
-//   CTA 0 ("S"): the 128 absorbed query rows live in TMEM (the A operand, 288
-//     columns); each 64-token block of the cache (9 pre-swizzled [64 x 64]
-//     chunks, 72 KB contiguous) arrives with one bulk copy into a ring of
-//     chunk slots, and S = Q K^T is formed by 36 tcgen05.mma (M=128,
-//     N=64, K=16) into one of two TMEM score buffers.  Eight warps (a query
-//     row's 64 scores split over two threads) run the online softmax in fp32,
-//     stage P (bf16) in shared memory, and one thread ships each P tile to
-//     CTA 1 with a single asynchronous bulk copy over DSMEM.
+//   CTA 0 ("S"): the latent part of the 128 absorbed query rows lives in TMEM
+//     (the A operand, 256 columns of packed bf16 pairs), the RoPE part in shared
+//     memory.  Each 128-token cache block (9 pre-swizzled [128 x 64] chunks,
+//     144 KB) arrives as three 48 KB bulk copies into a ring of three copy slots
+//     (blocks are pulled into L2 several tiles ahead, so the ring's copies hit
+//     L2), and S = Q K^T is formed by 36 tcgen05.mma (M=128, N=128, K=16:
+//     full-rate shape) into one of two TMEM score buffers.  Eight warps (a query
+//     row's 128 scores split over two threads) run the online softmax in fp32
+//     and stage P (bf16) in shared memory; a sender warp ships each staged P
+//     tile to CTA 1 with a single bulk copy over DSMEM, so neither the copy nor
+//     CTA 1's progress ever holds up the softmax.
 //   CTA 1 ("O"): keeps the unnormalised latent output O[128 x 512] fp32 in its
-//     whole TMEM and accumulates O += P V with 8 tcgen05.mma (M=128, N=256,
-//     K=16) per tile; V is the first 512 columns of the same cache block (its
-//     first 64 KB, one bulk copy), read as an MN-major operand.
+//     whole TMEM and accumulates O += P V with 32 tcgen05.mma per tile (M=128,
+//     N=128 per pair of latent chunks, K=16); V is the first 512 columns of the
+//     same cache block (its first 128 KB, four 32 KB bulk copies into a ring of
+//     five stages, so loads run 1.25 tiles ahead), read as an MN-major operand.
 // O for 128 rows x 512 fp32 fills an SM's 256 KB of TMEM, hence the pair.
 //
 // The softmax keeps a stale running max: it only rescales when a tile's max
@@ -46,56 +50,64 @@ using namespace sm100;
 
 namespace tc {
 
-constexpr int kTile = 64;            // tokens per tile
+constexpr int kTile = kBlockTokens;  // tokens per tile = one cache block (128)
 constexpr int kRows = 128;           // query rows per CTA pair
-constexpr int kChunk = 64 * 64 * 2;  // [64 tokens x 64 columns] bf16 = 8 KB
+constexpr int kChunk = kTile * 128;  // [128 tokens x 64 columns] bf16 = 16 KB
 constexpr int kKvChunks = 9;         // 576 / 64
-constexpr int kVChunks = 8;          // 512 / 64
-constexpr int kRing = 24;            // S CTA: ring of 8 KB cache chunks (2.67 tiles)
-constexpr int kStagesO = 3;          // O CTA: whole-tile V stages
-constexpr int kPrefetchTiles = 4;    // S CTA: tiles pulled into L2 ahead of the ring
-constexpr int kPBytes = kRows * kTile * 2;       // 16 KB bf16 P tile
-constexpr int kMsgBytes = kPBytes + kRows * 4 + 16;  // P | alpha[128] | flag (+pad): one bulk copy
-constexpr int kMsgStride = 17408;    // 1024-aligned message slots in the O CTA
+constexpr int kCopyChunks = 3;       // chunks per bulk copy (48 KB)
+constexpr int kCopies = kKvChunks / kCopyChunks;  // S CTA: copies per tile
+constexpr int kCopyBytes = kCopyChunks * kChunk;
+constexpr int kRingSlots = 3;        // S CTA: ring of 48 KB copy slots (one tile)
+constexpr int kVChunksPerStage = 2;  // O CTA: a V stage = 2 chunks (32 KB) = one N=128 MMA column block
+constexpr int kVStageBytes = kVChunksPerStage * kChunk;
+constexpr int kVPerTile = 8 / kVChunksPerStage;  // V stages per tile (the 8 latent chunks)
+constexpr int kVStages = 5;          // O CTA: ring of V stages
+constexpr int kPrefetchTiles = 4;    // S CTA: blocks pulled into L2 ahead of the ring
+constexpr int kPBytes = kRows * kTile * 2;       // 32 KB bf16 P tile: two [128 x 64] swizzled atoms
+constexpr int kMsgBytes = kPBytes + kRows * 4;  // P | alpha[128] (per-row rescale factors): one bulk copy
+constexpr int kMsgStride = 33792;    // 1024-aligned message slots in the O CTA
 constexpr int kSoftWarps = 8;        // S CTA: two warps per TMEM lane quadrant
 constexpr int kSoftThreads = kSoftWarps * 32;
-constexpr int kWarpProducer = 8, kWarpMma = 9;
-constexpr int kThreads = 320;
+constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpSender = 10;
+constexpr int kThreads = 352;
+constexpr int kSyncThreads = kSoftThreads + 32;  // softmax warps + the sender warp
+// named barriers, S CTA: 1..4 the two warps of a TMEM lane quadrant; the rest over kSyncThreads
+constexpr uint32_t kNbFail = 6, kNbStaged = 7, kNbStageFree = 8;
 constexpr uint64_t kLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleLog2 = 8.0f;
+static_assert(kKvChunks % kCopyChunks == 0, "a tile is a whole number of copies");
+static_assert(kTile == 128, "the MMA N and the P layout assume 128-token tiles");
 
 // TMEM columns (512 allocated in each CTA)
-constexpr uint32_t kColQ = 0;     // S CTA: Q rows, 288 columns of packed bf16 pairs
-constexpr uint32_t kColS0 = 384;  // S CTA: two 64-column score buffers (384, 448)
-__device__ __forceinline__ uint32_t col_s(uint32_t sb) { return kColS0 + 64u * sb; }
+constexpr uint32_t kColQ = 0;     // S CTA: latent Q rows, 256 columns of packed bf16 pairs
+constexpr uint32_t kColS0 = 256;  // S CTA: two 128-column score buffers (256, 384)
+__device__ __forceinline__ uint32_t col_s(uint32_t sb) { return kColS0 + 128u * sb; }
 
 // shared memory, S CTA
-constexpr int kSOffRing = 0;                                  // 24 x 8 KB
-constexpr int kSOffStage = kRing * kChunk;                    // 2 x kMsgBytes (local P messages)
-constexpr int kSOffXchg = kSOffStage + 2 * kMsgBytes;         // [2][128] fp32 half-row maxima / sums
+constexpr int kSOffRing = 0;                                  // 4 x 48 KB
+constexpr int kSOffQR = kRingSlots * kCopyBytes;              // RoPE part of Q: [128 x 64] swizzled, 16 KB
+constexpr int kSOffStage = kSOffQR + kRows * 128;             // the P message being built (kMsgBytes)
+constexpr int kSOffXchg = kSOffStage + kMsgStride;            // [2][128] fp32 half-row maxima / sums
 constexpr int kSOffBar = kSOffXchg + 2 * kRows * 4;
-// barrier slots, S CTA: a tile's chunks arrive together (one or two bulk copies) on
-// kSBarTFull[tile % 3]; the ring is released in triples of chunks (a tile always
-// starts on a triple: 9 n mod 24 is a multiple of 3), three commits per tile.
-constexpr int kTilesInRing = 3;  // at most 3 tiles own ring slots at any time (24 / 9 rounded up)
-constexpr int kTriples = kRing / 3;
-constexpr int kSBarTFull = 0, kSBarEmpty = kTilesInRing, kSBarSFull = kSBarEmpty + kTriples,
-              kSBarSEmpty = kSBarSFull + 2, kSBarPEmpty = kSBarSEmpty + 2, kSBarQReady = kSBarPEmpty + 2,
-              kSBarFin = kSBarQReady + 1, kSNumBars = kSBarFin + 1;
+constexpr int kSBarFull = 0, kSBarEmpty = kRingSlots, kSBarSFull = 2 * kRingSlots, kSBarSEmpty = kSBarSFull + 2,
+              kSBarPEmpty = kSBarSEmpty + 2, kSBarQReady = kSBarPEmpty + 2, kSBarFin = kSBarQReady + 1,
+              kSNumBars = kSBarFin + 1;
 constexpr int kSOffTail = kSOffBar + kSNumBars * 8;
 // shared memory, O CTA
-constexpr int kOOffV = 0;                                     // 3 x 8 x 8 KB
-constexpr int kOOffMsg = kStagesO * kVChunks * kChunk;        // 2 message slots
+constexpr int kOOffV = 0;                                     // 5 x 32 KB
+constexpr int kOOffMsg = kVStages * kVStageBytes;             // 2 message slots
 constexpr int kOOffBar = kOOffMsg + 2 * kMsgStride;
-constexpr int kOBarVFull = 0, kOBarVEmpty = kStagesO, kOBarPFull = 2 * kStagesO, kOBarOFull = kOBarPFull + 2,
+constexpr int kOBarVFull = 0, kOBarVEmpty = kVStages, kOBarPFull = 2 * kVStages, kOBarOFull = kOBarPFull + 2,
               kOBarOFree = kOBarOFull + 1, kOBarRescReq = kOBarOFree + 1, kOBarRescDone = kOBarRescReq + 1,
               kOBarODrain = kOBarRescDone + 1, kOBarFin = kOBarODrain + 1, kONumBars = kOBarFin + 1;
 constexpr int kOOffTail = kOOffBar + kONumBars * 8;
 constexpr int kTailBytes = 32;  // tmem base, abort flag, resc slot, tile total
 constexpr int kSmemBytes = (kSOffTail > kOOffTail ? kSOffTail : kOOffTail) + kTailBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kSOffStage % 16 == 0 && kMsgBytes % 16 == 0, "bulk copy alignment");
-static_assert(kOOffMsg % 1024 == 0 && kMsgStride % 1024 == 0, "P tiles must be 1024-byte aligned");
+static_assert(kSOffQR % 1024 == 0 && kSOffStage % 1024 == 0 && kOOffMsg % 1024 == 0 && kMsgStride % 1024 == 0,
+              "swizzle atoms 1024-aligned");
+static_assert(kMsgBytes % 16 == 0, "bulk copy size");
+static_assert(kMsgStride >= kMsgBytes, "message slot");
 
 struct Params {
     const uint16_t* q;
@@ -167,10 +179,10 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, uint32_t p
     if (dev_status) atomicOr(dev_status, MLA_DEVERR_TIMEOUT);
 }
 
-__device__ __forceinline__ float fmax32(const float (&v)[32]) {
+__device__ __forceinline__ float fmax64(const float (&v)[64]) {
     float a = fmaxf(v[0], v[1]), b = fmaxf(v[2], v[3]), c = fmaxf(v[4], v[5]), d = fmaxf(v[6], v[7]);
 #pragma unroll
-    for (int k = 8; k < 32; k += 4) {
+    for (int k = 8; k < 64; k += 4) {
         a = fmaxf(a, v[k]);
         b = fmaxf(b, v[k + 1]);
         c = fmaxf(c, v[k + 2]);
@@ -200,8 +212,10 @@ decode_tc_kernel(const Params p) {
     }
     if (tid == 0) {
         if (rank == 0) {
-            for (int i = 0; i < kTilesInRing; ++i) mbar_init(&bars[kSBarTFull + i], 1);
-            for (int i = 0; i < kTriples; ++i) mbar_init(&bars[kSBarEmpty + i], 1);
+            for (int i = 0; i < kRingSlots; ++i) {
+                mbar_init(&bars[kSBarFull + i], 1);
+                mbar_init(&bars[kSBarEmpty + i], 1);
+            }
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&bars[kSBarSFull + i], 1);
                 mbar_init(&bars[kSBarSEmpty + i], kSoftThreads);
@@ -210,7 +224,7 @@ decode_tc_kernel(const Params p) {
             mbar_init(&bars[kSBarQReady], kSoftThreads);
             mbar_init(&bars[kSBarFin], 1);
         } else {
-            for (int i = 0; i < kStagesO; ++i) {
+            for (int i = 0; i < kVStages; ++i) {
                 mbar_init(&bars[kOBarVFull + i], 1);
                 mbar_init(&bars[kOBarVEmpty + i], 1);
             }
@@ -260,10 +274,9 @@ decode_tc_kernel(const Params p) {
     if (active && rank == 0) {
         // =============================================================== S CTA
         if (warp == kWarpProducer) {
-            // ---- copy producer: each 64-token block (72 KB, already in the operand layout)
-            //      lands in the 24-slot ring with one bulk copy (two when it wraps the ring
-            //      end: 6 + 3 or 3 + 6 chunks).  A second walker pulls blocks kPrefetchTiles
-            //      ahead into L2.
+            // ---- copy producer: each 128-token block (144 KB, already in the operand layout)
+            //      lands as three 48 KB bulk copies, one per ring slot.  A second walker
+            //      pulls whole blocks kPrefetchTiles ahead into L2.
             if (lane == 0) {
                 SegWalk w, wp;
                 w.init(p, lo, hi, pidx);
@@ -280,73 +293,73 @@ decode_tc_kernel(const Params p) {
                     }
                 };
                 for (int i = 0; i < kPrefetchTiles; ++i) prefetch_one();
-                uint32_t n = 0;  // tiles issued
+                uint32_t nc = 0;  // copies issued
                 bool ok = true;
                 while (ok && w.next(p, s)) {
-                    for (int t = s.t0; ok && t < s.t1; ++t, ++n) {
+                    for (int t = s.t0; ok && t < s.t1; ++t) {
                         prefetch_one();
-                        const uint32_t gc = n * kKvChunks, s0 = gc % kRing;
-                        for (int c = 0; ok && c < 3; ++c) {
-                            const uint32_t g3 = gc / 3 + c;  // triple counter
-                            ok = mbar_wait(&bars[kSBarEmpty + g3 % kTriples], ((g3 / kTriples) & 1u) ^ 1u, abort_flag,
-                                           kLimitNs);
-                        }
-                        if (!ok) break;
-                        uint64_t* tb = &bars[kSBarTFull + n % kTilesInRing];
-                        mbar_arrive_expect_tx(tb, kKvChunks * kChunk);
                         const uint8_t* src = p.cache + (s.blk0 + t) * kBlockBytes;
-                        const uint32_t dst = sbase + kSOffRing + s0 * kChunk;
-                        if (s0 + kKvChunks <= static_cast<uint32_t>(kRing)) {
-                            bulk_load(dst, src, kKvChunks * kChunk, tb);
-                        } else {
-                            const uint32_t first = kRing - s0;  // chunks up to the ring end
-                            bulk_load(dst, src, first * kChunk, tb);
-                            bulk_load(sbase + kSOffRing, src + first * kChunk, (kKvChunks - first) * kChunk, tb);
+                        for (int k = 0; k < kCopies; ++k, ++nc) {
+                            const uint32_t slot = nc % kRingSlots, u = nc / kRingSlots;
+                            ok = mbar_wait(&bars[kSBarEmpty + slot], (u & 1u) ^ 1u, abort_flag, kLimitNs);
+                            if (!ok) break;
+                            mbar_arrive_expect_tx(&bars[kSBarFull + slot], kCopyBytes);
+                            bulk_load(sbase + kSOffRing + slot * kCopyBytes, src + k * kCopyBytes, kCopyBytes,
+                                      &bars[kSBarFull + slot]);
                         }
                     }
                 }
                 if (!ok) raise_abort(abort_flag, peer_abort, p.dev_status);
                 // let every issued copy land before the CTA can exit
-                for (uint32_t i = (n > kTilesInRing ? n - kTilesInRing : 0); i < n; ++i)
-                    mbar_wait(&bars[kSBarTFull + i % kTilesInRing], (i / kTilesInRing) & 1u, &never, kLimitNs);
+                for (uint32_t i = (nc > kRingSlots ? nc - kRingSlots : 0); i < nc; ++i)
+                    mbar_wait(&bars[kSBarFull + i % kRingSlots], (i / kRingSlots) & 1u, &never, kLimitNs);
             }
         } else if (warp == kWarpMma) {
-            // ---- MMA issuer (one thread): S[sb] = Q K^T, A from TMEM, B = cache chunks
-            //      (K-major SW128).  Once a tile has landed its 36 MMAs go out back to back;
-            //      each triple of ring slots is released (commit) once its 12 MMAs finish.
+            // ---- MMA issuer (one thread): S[sb] = Q K^T.  Latent chunks: A from TMEM; the
+            //      RoPE chunk: A = Q^R in shared memory.  B = cache chunks (K-major SW128,
+            //      128 rows).  Each ring slot is released (commit) once its 12 MMAs finish.
             if (lane == 0) {
                 constexpr uint32_t idesc = idesc_bf16_f32(kRows, kTile, false, false);
                 const uint64_t ring_desc = sdesc_sw128(sbase + kSOffRing, 16, 1024);
+                const uint64_t qr_desc = sdesc_sw128(sbase + kSOffQR, 16, 1024);
                 SegWalk w;
                 w.init(p, lo, hi, pidx);
                 Seg s;
-                uint32_t n = 0, kseg = 0, gc = 0;
+                uint32_t n = 0, kseg = 0, nc = 0;
                 bool ok = true;
                 while (ok && w.next(p, s)) {
                     ok = mbar_wait(&bars[kSBarQReady], kseg & 1u, abort_flag, kLimitNs);
                     ++kseg;
-                    for (int t = s.t0; ok && t < s.t1; ++t, ++n, gc += kKvChunks) {
+                    for (int t = s.t0; ok && t < s.t1; ++t, ++n) {
                         const uint32_t sb = n & 1u, us = n >> 1;
-                        ok = mbar_wait(&bars[kSBarSEmpty + sb], (us & 1u) ^ 1u, abort_flag, kLimitNs) &&
-                             mbar_wait(&bars[kSBarTFull + n % kTilesInRing], (n / kTilesInRing) & 1u, abort_flag,
-                                       kLimitNs);
-                        if (!ok) break;
-                        tc_fence_after();
+                        ok = mbar_wait(&bars[kSBarSEmpty + sb], (us & 1u) ^ 1u, abort_flag, kLimitNs);
                         const uint32_t d = tmem + col_s(sb);
-                        const uint32_t s0 = gc % kRing;
+                        for (int k = 0; ok && k < kCopies; ++k, ++nc) {
+                            const uint32_t slot = nc % kRingSlots, u = nc / kRingSlots;
+                            ok = mbar_wait(&bars[kSBarFull + slot], u & 1u, abort_flag, kLimitNs);
+                            if (!ok) break;
+                            tc_fence_after();
 #pragma unroll
-                        for (int c = 0; c < kKvChunks; ++c) {
-                            const uint32_t slot = (s0 + c) % kRing;
-                            const uint64_t cd = ring_desc + (static_cast<uint64_t>(slot) << 9);  // 8 KB / 16
-                            const uint32_t qa = tmem + kColQ + 32 * c;
-                            mma_ts(d, qa, cd, idesc, c ? 1u : 0u);
-                            mma_ts(d, qa + 8, cd + 2, idesc, 1u);
-                            mma_ts(d, qa + 16, cd + 4, idesc, 1u);
-                            mma_ts(d, qa + 24, cd + 6, idesc, 1u);
-                            if (c % 3 == 2)  // triple free once its 12 MMAs finish
-                                mma_commit(smem_u32(&bars[kSBarEmpty + ((gc / 3 + c / 3) % kTriples)]));
+                            for (int j = 0; j < kCopyChunks; ++j) {
+                                const int c = kCopyChunks * k + j;  // chunk of the block
+                                const uint64_t cd =
+                                    ring_desc + (static_cast<uint64_t>(slot * kCopyBytes + j * kChunk) >> 4);
+                                if (c < 8) {
+                                    const uint32_t qa = tmem + kColQ + 32 * c;
+                                    mma_ts(d, qa, cd, idesc, c ? 1u : 0u);
+                                    mma_ts(d, qa + 8, cd + 2, idesc, 1u);
+                                    mma_ts(d, qa + 16, cd + 4, idesc, 1u);
+                                    mma_ts(d, qa + 24, cd + 6, idesc, 1u);
+                                } else {
+                                    mma_ss(d, qr_desc, cd, idesc, 1u);
+                                    mma_ss(d, qr_desc + 2, cd + 2, idesc, 1u);
+                                    mma_ss(d, qr_desc + 4, cd + 4, idesc, 1u);
+                                    mma_ss(d, qr_desc + 6, cd + 6, idesc, 1u);
+                                }
+                            }
+                            mma_commit(smem_u32(&bars[kSBarEmpty + slot]));
                         }
-                        mma_commit(smem_u32(&bars[kSBarSFull + sb]));
+                        if (ok) mma_commit(smem_u32(&bars[kSBarSFull + sb]));
                     }
                 }
                 if (!ok) raise_abort(abort_flag, peer_abort, p.dev_status);
@@ -354,15 +367,16 @@ decode_tc_kernel(const Params p) {
                 mbar_wait(&bars[kSBarFin], 0, &never, kLimitNs);
             }
             __syncwarp();
-        } else {
+        } else if (warp < kSoftWarps) {
             // ---- softmax: 8 warps; warp (q, hf) owns TMEM lanes 32q.. (query rows) and
-            //      score columns 32hf .. 32hf + 31 of each 64-token tile
+            //      score columns 64hf .. 64hf + 63 of each 128-token tile
             const int qd = warp & 3, hf = warp >> 2;
             const int r = 32 * qd + lane;
             const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * qd) << 16);
             float* xchg = reinterpret_cast<float*>(smem + kSOffXchg);  // [2][128]
-            const uint32_t peer_msg = mapa(sbase + kOOffMsg, peer);
-            const uint32_t peer_pfull = mapa(sbase + kOOffBar + kOBarPFull * 8, peer);
+            // this thread's row of P in the staged message: atom hf, row r (8 swizzled units)
+            uint8_t* stage = smem + kSOffStage;
+            uint8_t* prow = stage + hf * (kRows * 128) + r * 128;
             const int rr = g * kRows + r;
             const bool row_ok = rr < p.R;
             const int j = row_ok ? rr / p.H : 0;
@@ -375,8 +389,9 @@ decode_tc_kernel(const Params p) {
             while (!failed && have) {
                 wn = w;
                 const bool have_next = wn.next(p, sn);
-                // this segment's absorbed query row -> TMEM columns 0..287 (warp hf=0: chunks 0..4,
-                // hf=1: chunks 5..8); the next segment's rows are prefetched into L2
+                // this segment's absorbed query row: latent part -> TMEM columns 0..255 (warp
+                // hf=0: columns 0..127, hf=1: 128..255), RoPE part -> shared memory row r
+                // (hf=0: units 0..3, hf=1: units 4..7).  The next segment's row goes to L2.
                 const uint16_t* qrow = p.q + (static_cast<int64_t>(s.b) * p.R + (row_ok ? rr : 0)) * kRow;
                 if (have_next && row_ok) {
                     const char* nq = reinterpret_cast<const char*>(p.q + (static_cast<int64_t>(sn.b) * p.R + rr) * kRow);
@@ -384,22 +399,28 @@ decode_tc_kernel(const Params p) {
                 }
                 __syncwarp();
                 {
-                    const int c0 = hf ? 5 : 0, c1 = hf ? 9 : 5;
-                    for (int c = c0; c < c1; c += 2) {
+                    const uint4* src = reinterpret_cast<const uint4*>(qrow);
+#pragma unroll 1
+                    for (int c = 4 * hf; c < 4 * hf + 4; c += 2) {
                         uint32_t v0[32], v1[32];
-                        const uint4* src = reinterpret_cast<const uint4*>(qrow + 64 * c);
-                        const bool two = (c + 1) < c1;
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
-                            const uint4 x = row_ok ? src[k] : make_uint4(0, 0, 0, 0);
-                            const uint4 y = (row_ok && two) ? src[k + 8] : make_uint4(0, 0, 0, 0);
+                            const uint4 x = row_ok ? src[8 * c + k] : make_uint4(0, 0, 0, 0);
+                            const uint4 y = row_ok ? src[8 * c + 8 + k] : make_uint4(0, 0, 0, 0);
                             v0[4 * k] = x.x; v0[4 * k + 1] = x.y; v0[4 * k + 2] = x.z; v0[4 * k + 3] = x.w;
                             v1[4 * k] = y.x; v1[4 * k + 1] = y.y; v1[4 * k + 2] = y.z; v1[4 * k + 3] = y.w;
                         }
                         tmem_st32(t_lane + kColQ + 32 * c, v0);
-                        if (two) tmem_st32(t_lane + kColQ + 32 * (c + 1), v1);
+                        tmem_st32(t_lane + kColQ + 32 * (c + 1), v1);
+                    }
+                    uint8_t* qr = smem + kSOffQR + r * 128;
+#pragma unroll
+                    for (int u = 4 * hf; u < 4 * hf + 4; ++u) {
+                        const uint4 x = row_ok ? src[64 + u] : make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4*>(qr + ((u ^ (r & 7)) << 4)) = x;
                     }
                 }
+                fence_proxy_async_cta();
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bars[kSBarQReady]);
@@ -410,23 +431,27 @@ decode_tc_kernel(const Params p) {
                     bool ok = mbar_wait(&bars[kSBarSFull + sb], us & 1u, abort_flag, kLimitNs);
                     __syncwarp();
                     tc_fence_after();
-                    float sv[32];
+                    float sv[64];
                     {
-                        uint32_t a[32];
-                        tmem_ld32(t_lane + col_s(sb) + 32 * hf, a);
+                        uint32_t a[32], b[32];
+                        tmem_ld32(t_lane + col_s(sb) + 64 * hf, a);
+                        tmem_ld32(t_lane + col_s(sb) + 64 * hf + 32, b);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) sv[k] = __uint_as_float(a[k]);
+                        for (int k = 0; k < 32; ++k) {
+                            sv[k] = __uint_as_float(a[k]);
+                            sv[32 + k] = __uint_as_float(b[k]);
+                        }
                     }
                     tc_fence_before();
                     mbar_arrive(&bars[kSBarSEmpty + sb]);
-                    const int nvalid = lim - t * kTile - 32 * hf;  // columns < nvalid are visible
-                    if (nvalid < 32) {
+                    const int nvalid = lim - t * kTile - 64 * hf;  // columns < nvalid are visible
+                    if (nvalid < 64) {
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) sv[k] = k < nvalid ? sv[k] : -CUDART_INF_F;
+                        for (int k = 0; k < 64; ++k) sv[k] = k < nvalid ? sv[k] : -CUDART_INF_F;
                     }
                     // row max over both halves (raw scores; the scale is positive)
-                    xchg[hf * kRows + r] = fmax32(sv);
+                    xchg[hf * kRows + r] = fmax64(sv);
                     bar_sync(1 + qd, 64);
                     const float tmax = fmaxf(xchg[r], xchg[kRows + r]) * p.scale_log2;
                     const bool resc = tmax > m + kRescaleLog2;
@@ -437,48 +462,30 @@ decode_tc_kernel(const Params p) {
                         m = tmax;
                     }
                     const float mneg = (m == -CUDART_INF_F) ? 0.f : -m;
-                    uint32_t pk[16];
+                    uint32_t pk[32];
                     float lsum = 0.f;
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
+                    for (int k = 0; k < 32; ++k) {
                         const float p0 = ex2_approx(fmaf(sv[2 * k], p.scale_log2, mneg));
                         const float p1 = ex2_approx(fmaf(sv[2 * k + 1], p.scale_log2, mneg));
                         lsum += p0 + p1;
                         pk[k] = cvt_bf16x2(p0, p1);
                     }
                     l += lsum;
-                    // staging slot sb is free once the bulk copy of two tiles ago has read it
-                    if (tid == 0 && n >= 2) bulk_wait_group_read<1>();
-                    const bool flag = bar_red_or(5, kSoftThreads, resc && t != s.t0);
-                    uint8_t* msg = smem + kSOffStage + sb * kMsgBytes;
-                    {
-                        // P row r, columns 32hf.. : 16-byte units 4hf..4hf+3, 128-byte swizzle
-                        uint8_t* prow = msg + r * 128;
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int uu = 4 * hf + u;
-                            *reinterpret_cast<uint4*>(prow + ((uu ^ (r & 7)) << 4)) =
-                                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-                        }
-                        if (hf == 0) reinterpret_cast<float*>(msg + kPBytes)[r] = alpha;
-                        if (tid == 0) *reinterpret_cast<uint32_t*>(msg + kPBytes + kRows * 4) = flag ? 1u : 0u;
-                    }
-                    fence_proxy_async_cta();
-                    if (bar_red_or(6, kSoftThreads, !ok || *abort_flag != 0)) {
+                    if (bar_red_or(kNbFail, kSyncThreads, !ok || *abort_flag != 0)) {
                         failed = true;
                         break;
                     }
-                    if (tid == 0) {
-                        // ship the message once the O CTA has finished with this slot
-                        if (mbar_wait<true>(&bars[kSBarPEmpty + sb], (us & 1u) ^ 1u, abort_flag, kLimitNs)) {
-                            mbar_arrive_expect_tx_remote(peer_pfull + 8 * sb, kMsgBytes);
-                            bulk_copy_to_peer(peer_msg + sb * kMsgStride, sbase + kSOffStage + sb * kMsgBytes, kMsgBytes,
-                                              peer_pfull + 8 * sb);
-                            bulk_commit_group();
-                        } else {
-                            raise_abort(abort_flag, peer_abort, p.dev_status);
-                        }
-                    }
+                    // the sender has seen the previous tile's copy read the staging buffer
+                    bar_sync(kNbStageFree, kSyncThreads);
+                    // P row r, columns 64hf.. -> atom hf, row r: 16-byte units u at (u ^ (r % 8))
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) =
+                            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                    if (hf == 0) reinterpret_cast<float*>(stage + kPBytes)[r] = alpha;
+                    fence_proxy_async_cta();
+                    bar_arrive(kNbStaged, kSyncThreads);
                 }
                 if (failed) break;
                 // segment result: (m, l) with l summed over both column halves
@@ -492,59 +499,101 @@ decode_tc_kernel(const Params p) {
                 have = have_next;
             }
             if (failed && tid == 0) raise_abort(abort_flag, peer_abort, p.dev_status);
-            if (tid == 0) bulk_wait_group_read<0>();
+        } else if (warp == kWarpSender) {
+            // ---- sender: ships each staged P tile (one bulk copy, completing on the O CTA's
+            //      barrier) once the O CTA has released that message slot.  Takes the same
+            //      per-tile barrier steps as the softmax warps.
+            const uint32_t peer_msg = mapa(sbase + kOOffMsg, peer);
+            const uint32_t peer_pfull = mapa(sbase + kOOffBar + kOBarPFull * 8, peer);
+            SegWalk w;
+            w.init(p, lo, hi, pidx);
+            Seg s;
+            uint32_t n = 0;
+            bool failed = false;
+            while (!failed && w.next(p, s)) {
+                for (int t = s.t0; t < s.t1; ++t, ++n) {
+                    const uint32_t pb = n & 1u, up = n >> 1;
+                    if (bar_red_or(kNbFail, kSyncThreads, *abort_flag != 0)) {
+                        failed = true;
+                        break;
+                    }
+                    if (lane == 0) bulk_wait_group_read<0>();
+                    __syncwarp();
+                    bar_arrive(kNbStageFree, kSyncThreads);
+                    bar_sync(kNbStaged, kSyncThreads);
+                    if (lane == 0) {
+                        if (mbar_wait<true>(&bars[kSBarPEmpty + pb], (up & 1u) ^ 1u, abort_flag, kLimitNs)) {
+                            mbar_arrive_expect_tx_remote(peer_pfull + 8 * pb, kMsgBytes);
+                            bulk_copy_to_peer(peer_msg + pb * kMsgStride, sbase + kSOffStage, kMsgBytes,
+                                              peer_pfull + 8 * pb);
+                            bulk_commit_group();
+                        } else {
+                            raise_abort(abort_flag, peer_abort, p.dev_status);
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
         }
     } else if (active && rank == 1) {
         // =============================================================== O CTA
         if (warp == kWarpProducer) {
-            // ---- copy producer: the 8 latent chunks of each block (its first 64 KB) = V
+            // ---- copy producer: the 8 latent chunks of each block (its first 128 KB) = V,
+            //      as four bulk copies of 2 chunks into the ring of V stages
             if (lane == 0) {
                 SegWalk w;
                 w.init(p, lo, hi, pidx);
                 Seg s;
-                uint32_t n = 0;
+                uint32_t nv = 0;  // stage loads issued
                 bool ok = true;
                 while (ok && w.next(p, s)) {
-                    for (int t = s.t0; t < s.t1; ++t, ++n) {
-                        const uint32_t st = n % kStagesO, u = n / kStagesO;
-                        if (!mbar_wait(&bars[kOBarVEmpty + st], (u & 1u) ^ 1u, abort_flag, kLimitNs)) {
-                            ok = false;
-                            break;
+                    for (int t = s.t0; ok && t < s.t1; ++t) {
+                        const uint8_t* src = p.cache + (s.blk0 + t) * kBlockBytes;
+                        for (int k = 0; k < kVPerTile; ++k, ++nv) {
+                            const uint32_t st = nv % kVStages, u = nv / kVStages;
+                            if (!mbar_wait(&bars[kOBarVEmpty + st], (u & 1u) ^ 1u, abort_flag, kLimitNs)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(&bars[kOBarVFull + st], kVStageBytes);
+                            bulk_load(sbase + kOOffV + st * kVStageBytes, src + k * kVStageBytes, kVStageBytes,
+                                      &bars[kOBarVFull + st]);
                         }
-                        mbar_arrive_expect_tx(&bars[kOBarVFull + st], kVChunks * kChunk);
-                        bulk_load(sbase + kOOffV + st * kVChunks * kChunk, p.cache + (s.blk0 + t) * kBlockBytes,
-                                  kVChunks * kChunk, &bars[kOBarVFull + st]);
                     }
                 }
                 if (!ok) raise_abort(abort_flag, peer_abort, p.dev_status);
-                for (uint32_t i = (n > kStagesO ? n - kStagesO : 0); i < n; ++i)
-                    mbar_wait(&bars[kOBarVFull + i % kStagesO], (i / kStagesO) & 1u, &never, kLimitNs);
+                for (uint32_t i = (nv > kVStages ? nv - kVStages : 0); i < nv; ++i)
+                    mbar_wait(&bars[kOBarVFull + i % kVStages], (i / kVStages) & 1u, &never, kLimitNs);
             }
         } else if (warp == kWarpMma) {
-            // ---- MMA issuer (one thread): O += P V (A = P, K-major SW128; B = V, MN-major SW128)
-            constexpr uint32_t idesc = idesc_bf16_f32(kRows, 256, false, true);
+            // ---- MMA issuer (one thread): O += P V (A = P, K-major SW128; B = V, MN-major SW128
+            //      with 16 KB between 64-column atoms)
+            constexpr uint32_t idesc = idesc_bf16_f32(kRows, 128, false, true);
             const uint32_t peer_pempty = mapa(sbase + kSOffBar + kSBarPEmpty * 8, peer);
             const uint64_t p_desc = sdesc_sw128(sbase + kOOffMsg, 16, 1024);
             const uint64_t v_desc = sdesc_sw128(sbase + kOOffV, kChunk, 1024);
             SegWalk w;
             w.init(p, lo, hi, pidx);
             Seg s;
-            uint32_t n = 0, kseg = 0, nresc = 0;
+            uint32_t n = 0, nv = 0, kseg = 0, nresc = 0;
             bool ok = true;
             while (ok && w.next(p, s)) {
                 for (int t = s.t0; ok && t < s.t1; ++t, ++n) {
-                    const uint32_t st = n % kStagesO, u = n / kStagesO;
                     const uint32_t pb = n & 1u, up = n >> 1;
                     const bool first = (t == s.t0);
                     if (lane == 0) {
-                        ok = mbar_wait(&bars[kOBarVFull + st], u & 1u, abort_flag, kLimitNs) &&
-                             mbar_wait<true>(&bars[kOBarPFull + pb], up & 1u, abort_flag, kLimitNs);
+                        ok = mbar_wait<true>(&bars[kOBarPFull + pb], up & 1u, abort_flag, kLimitNs);
                         if (ok && first) ok = mbar_wait(&bars[kOBarOFree], (kseg & 1u) ^ 1u, abort_flag, kLimitNs);
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     const uint8_t* msg = smem + kOOffMsg + pb * kMsgStride;
-                    if (!first && *reinterpret_cast<const volatile uint32_t*>(msg + kPBytes + kRows * 4) != 0u) {
+                    // some row's stale max moved iff its alpha is not exactly 1
+                    const float4 al = reinterpret_cast<const float4*>(msg + kPBytes)[lane];
+                    const bool resc = __any_sync(0xffffffffu, al.x != 1.f || al.y != 1.f || al.z != 1.f || al.w != 1.f);
+                    if (!first && resc) {
                         // stale max moved: have the epilogue rescale O once all earlier MMAs are done
                         if (lane == 0) {
                             *resc_pb = static_cast<int>(pb);
@@ -557,31 +606,39 @@ decode_tc_kernel(const Params p) {
                         if (!ok) break;
                     }
                     const int nvalid = min(kTile, s.L - t * kTile);
-                    if (nvalid < kTile) {
-                        // rows past the sequence end: P is 0 there, make V 0 too (no 0 * NaN)
-                        uint8_t* vst = smem + kOOffV + st * kVChunks * kChunk;
-                        const int nz = (kTile - nvalid) * 8;  // 16-byte units per chunk
-                        for (int i = lane; i < kVChunks * nz; i += 32) {
-                            const int c = i / nz, k = i % nz;
-                            *reinterpret_cast<uint4*>(vst + c * kChunk + nvalid * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+                    for (int k = 0; k < kVPerTile; ++k, ++nv) {
+                        const uint32_t st = nv % kVStages, u = nv / kVStages;
+                        if (lane == 0) ok = mbar_wait(&bars[kOBarVFull + st], u & 1u, abort_flag, kLimitNs);
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        if (!ok) break;
+                        constexpr int nch = kVChunksPerStage;
+                        uint8_t* vst = smem + kOOffV + st * kVStageBytes;
+                        if (nvalid < kTile) {
+                            // rows past the sequence end: P is 0 there, make V 0 too (no 0 * NaN)
+                            const int nz = (kTile - nvalid) * 8;  // 16-byte units per chunk
+                            for (int i = lane; i < nch * nz; i += 32) {
+                                const int c = i / nz, q = i % nz;
+                                *reinterpret_cast<uint4*>(vst + c * kChunk + nvalid * 128 + q * 16) =
+                                    make_uint4(0, 0, 0, 0);
+                            }
                         }
+                        // V may have been zeroed by this warp: order that before the tensor core reads
                         fence_proxy_async_cta();
                         __syncwarp();
-                    }
-                    if (lane == 0) {
-                        tc_fence_after();
-                        const uint64_t pd = p_desc + (static_cast<uint64_t>(pb * kMsgStride) >> 4);
-                        const uint64_t vd = v_desc + (static_cast<uint64_t>(st * kVChunks * kChunk) >> 4);
+                        if (lane == 0) {
+                            tc_fence_after();
+                            const uint64_t vd = v_desc + (static_cast<uint64_t>(st * kVStageBytes) >> 4);
+                            const uint64_t pd = p_desc + (static_cast<uint64_t>(pb * kMsgStride) >> 4);
 #pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                            for (int k = 0; k < kTile / 16; ++k)
-                                mma_ss(tmem + 256 * half, pd + 2 * k, vd + ((4 * half * kChunk + k * 2048) >> 4), idesc,
-                                       (first && k == 0) ? 0u : 1u);
+                            for (int kk = 0; kk < kTile / 16; ++kk)
+                                mma_ss(tmem + 128 * k, pd + (((kk >> 2) * kRows * 128 + (kk & 3) * 32) >> 4),
+                                       vd + ((kk * 2048) >> 4), idesc, (first && kk == 0) ? 0u : 1u);
+                            mma_commit(smem_u32(&bars[kOBarVEmpty + st]));
                         }
-                        mma_commit(smem_u32(&bars[kOBarVEmpty + st]));
-                        mma_commit(peer_pempty + 8 * pb);
+                        __syncwarp();
                     }
+                    if (!ok) break;
+                    if (lane == 0) mma_commit(peer_pempty + 8 * pb);
                     __syncwarp();
                 }
                 if (!ok) break;

@@ -16,12 +16,13 @@ constexpr int kRow = kDc + kDr;    // packed cache row (576 bf16 = 1152 B)
 constexpr int kMaxHeads = 128;
 constexpr int kMaxNq = 16;
 constexpr int kBlockTokens = MLA_BLOCK_TOKENS;  // tokens per cache block
-constexpr int kBlockBytes = MLA_BLOCK_BYTES;    // 9 chunks x [64 rows x 128 B]
-static_assert(kBlockBytes == 9 * kBlockTokens * 128, "block layout");
+constexpr int kBlockBytes = MLA_BLOCK_BYTES;    // 9 chunks x [128 rows x 128 B]
+constexpr int kBlockChunk = kBlockTokens * 128;  // bytes of one 64-column chunk of a block
+static_assert(kBlockBytes == 9 * kBlockChunk, "block layout");
 
 // Byte offset of column c of row r inside a cache block (128-byte swizzle per 64-column chunk).
 __host__ __device__ __forceinline__ int block_offset(int r, int c) {
-    return (c >> 6) * 8192 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2;
+    return (c >> 6) * kBlockChunk + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2;
 }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {

@@ -239,6 +239,22 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+// Asynchronous stores into a peer CTA's shared memory (address from mapa); each completes its
+// byte count on the peer's mbarrier `bar` (also from mapa).  Stores issued this way are ordered
+// for the peer's tensor-core reads by a fence.proxy.async on the peer after its barrier wait.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     addr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t v, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+                 "r"(bar)
+                 : "memory");
+}
+
 // Named barrier over `nthreads` threads with an OR reduction of `pred`.
 __device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t nthreads, bool pred) {
     uint32_t out;
@@ -255,6 +271,9 @@ __device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t nthreads, bool 
 
 __device__ __forceinline__ void bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint32_t id, uint32_t nthreads) {
+    asm volatile("barrier.cta.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ----------------------------------------------------------------- tcgen05

@@ -13,14 +13,14 @@ import mla_latent_kv_34_b200 as mla
 from oracle import naive as on
 
 NAN_BF16 = 0x7FC0  # quiet NaN pattern put in cache rows no sequence owns
-BLOCK_TOKENS, BLOCK_BYTES = 64, 73728
+BLOCK_TOKENS, BLOCK_BYTES = 128, 147456
 
 
 def _block_index_map() -> np.ndarray:
-    """[64, 576] uint16 offsets inside a cache block of (row r, column c), per the mla.h layout."""
-    r = np.arange(64)[:, None]
+    """[128, 576] uint16 offsets inside a cache block of (row r, column c), per the mla.h layout."""
+    r = np.arange(BLOCK_TOKENS)[:, None]
     c = np.arange(576)[None, :]
-    byte = (c // 64) * 8192 + r * 128 + ((((c % 64) // 8) ^ (r % 8)) * 16) + (c % 8) * 2
+    byte = (c // 64) * (BLOCK_TOKENS * 128) + r * 128 + ((((c % 64) // 8) ^ (r % 8)) * 16) + (c % 8) * 2
     return (byte // 2).astype(np.int64)
 
 

@@ -76,10 +76,10 @@ def test_append_bit_exact_with_canary(cuda_ok, H):
     # logical rows from the oracle's fp32 emulation, placed per the documented block layout
     rows = np.concatenate([c, oapp.rotate_k_bits(k, pos)], axis=1)
     expect = canary.copy()
-    blk = seq_block[seq_idx] + pos // 64
-    H.pack_rows(expect, blk, pos % 64, rows)
+    blk = seq_block[seq_idx] + pos // H.BLOCK_TOKENS
+    H.pack_rows(expect, blk, pos % H.BLOCK_TOKENS, rows)
     got = H.cache_u16(cache)
-    np.testing.assert_array_equal(H.unpack_rows(got, blk, pos % 64), rows)
+    np.testing.assert_array_equal(H.unpack_rows(got, blk, pos % H.BLOCK_TOKENS), rows)
     np.testing.assert_array_equal(got, expect)
 
 
@@ -88,7 +88,7 @@ def test_append_large_positions_bit_exact(cuda_ok, H):
     dev = "cuda"
     T = 512
     pos = (131071 - 255 * (T - 1 - np.arange(T, dtype=np.int64))).astype(np.int32)
-    cap_blocks = int(pos.max()) // 64 + 1
+    cap_blocks = int(pos.max()) // H.BLOCK_TOKENS + 1
     cache = mla.new_cache(cap_blocks, dev)
     c = mi.normal_bf16(78, 1, 0, T * 512).reshape(T, 512)
     k = mi.normal_bf16(78, 2, 0, T * 64).reshape(T, 64)
@@ -96,7 +96,7 @@ def test_append_large_positions_bit_exact(cuda_ok, H):
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     mla.append_cache(cache, torch.zeros(1, dtype=torch.int64, device=dev), torch.zeros(T, dtype=torch.int32, device=dev),
                      torch.from_numpy(pos).to(dev), H.to_dev_bf16(c, dev), H.to_dev_bf16(k, dev), tab, st)
-    got = H.unpack_rows(H.cache_u16(cache), pos // 64, pos % 64)
+    got = H.unpack_rows(H.cache_u16(cache), pos // H.BLOCK_TOKENS, pos % H.BLOCK_TOKENS)
     np.testing.assert_array_equal(got[:, :512], c)
     np.testing.assert_array_equal(got[:, 512:], oapp.rotate_k_bits(k, pos))
     assert int(st.item()) == 0
@@ -110,9 +110,9 @@ def test_append_out_of_range_is_reported_and_skipped(cuda_ok, H):
     c = torch.ones((2, 512), dtype=torch.bfloat16, device=dev)
     k = torch.ones((2, 64), dtype=torch.bfloat16, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    # sequence 1 starts at block 2: position 70 lands in block 3 = out of range
+    # sequence 1 starts at block 2: position 140 lands in block 3 = out of range
     mla.append_cache(cache, torch.tensor([0, 2], device=dev), torch.tensor([0, 1], dtype=torch.int32, device=dev),
-                     torch.tensor([3, 70], dtype=torch.int32, device=dev), c, k, tab, st)
+                     torch.tensor([3, 140], dtype=torch.int32, device=dev), c, k, tab, st)
     torch.cuda.synchronize()
     assert int(st.item()) & 0x1
     u = H.cache_u16(cache)
@@ -164,7 +164,8 @@ def test_decode_tiny_full(cuda_ok, H):
 
 
 @pytest.mark.parametrize("L,n_q,Hh", [(1, 1, 16), (2, 2, 16), (3, 2, 128), (64, 1, 128), (65, 2, 128),
-                                      (127, 1, 1), (200, 2, 100), (1000, 1, 64), (129, 2, 64)])
+                                      (127, 1, 1), (128, 1, 128), (200, 2, 100), (1000, 1, 64), (129, 2, 64),
+                                      (257, 2, 128)])
 def test_decode_edge_shapes(cuda_ok, H, L, n_q, Hh):
     cfg = mi.MLAConfig("edge", B=2, H=Hh, n_q=n_q, L=L, seed=1000 + L + Hh)
     prob = H.build_problem(cfg, lengths=[L, max(n_q, L // 2 + 1)])
