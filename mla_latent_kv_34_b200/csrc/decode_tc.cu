@@ -19,10 +19,11 @@
 //     tile to CTA 1 with a single bulk copy over DSMEM, so neither the copy nor
 //     CTA 1's progress ever holds up the softmax.
 //   CTA 1 ("O"): keeps the unnormalised latent output O[128 x 512] fp32 in its
-//     whole TMEM and accumulates O += P V with 32 tcgen05.mma per tile (M=128,
-//     N=128 per pair of latent chunks, K=16); V is the first 512 columns of the
-//     same cache block (its first 128 KB, four 32 KB bulk copies into a ring of
-//     five stages, so loads run 1.25 tiles ahead), read as an MN-major operand.
+//     whole TMEM and accumulates O += P V with 16 tcgen05.mma per tile (M=128,
+//     N=256 per four latent chunks, K=16: the widest N re-reads P least often
+//     from shared memory, whose bandwidth bounds this SM); V is the first 512
+//     columns of the same cache block (its first 128 KB, two 64 KB bulk copies
+//     into two stages), read as an MN-major operand.
 // O for 128 rows x 512 fp32 fills an SM's 256 KB of TMEM, hence the pair.
 //
 // The softmax keeps a stale running max: it only rescales when a tile's max
@@ -58,11 +59,11 @@ constexpr int kCopyChunks = 3;       // chunks per bulk copy (48 KB)
 constexpr int kCopies = kKvChunks / kCopyChunks;  // S CTA: copies per tile
 constexpr int kCopyBytes = kCopyChunks * kChunk;
 constexpr int kRingSlots = 3;        // S CTA: ring of 48 KB copy slots (one tile)
-constexpr int kVChunksPerStage = 2;  // O CTA: a V stage = 2 chunks (32 KB) = one N=128 MMA column block
+constexpr int kVChunksPerStage = 4;  // O CTA: a V stage = 4 chunks (64 KB) = one N=256 MMA column block
 constexpr int kVStageBytes = kVChunksPerStage * kChunk;
 constexpr int kVPerTile = 8 / kVChunksPerStage;  // V stages per tile (the 8 latent chunks)
-constexpr int kVStages = 5;          // O CTA: ring of V stages
-constexpr int kPrefetchTiles = 4;    // S CTA: blocks pulled into L2 ahead of the ring
+constexpr int kVStages = 2;          // O CTA: ring of V stages
+constexpr int kPrefetchTiles = 1;    // S CTA: blocks pulled into L2 ahead of the ring
 constexpr int kPBytes = kRows * kTile * 2;       // 32 KB bf16 P tile: two [128 x 64] swizzled atoms
 constexpr int kMsgBytes = kPBytes + kRows * 4;  // P | alpha[128] (per-row rescale factors): one bulk copy
 constexpr int kMsgStride = 33792;    // 1024-aligned message slots in the O CTA
@@ -94,14 +95,14 @@ constexpr int kSBarFull = 0, kSBarEmpty = kRingSlots, kSBarSFull = 2 * kRingSlot
               kSNumBars = kSBarFin + 1;
 constexpr int kSOffTail = kSOffBar + kSNumBars * 8;
 // shared memory, O CTA
-constexpr int kOOffV = 0;                                     // 5 x 32 KB
+constexpr int kOOffV = 0;                                     // 2 x 64 KB
 constexpr int kOOffMsg = kVStages * kVStageBytes;             // 2 message slots
 constexpr int kOOffBar = kOOffMsg + 2 * kMsgStride;
 constexpr int kOBarVFull = 0, kOBarVEmpty = kVStages, kOBarPFull = 2 * kVStages, kOBarOFull = kOBarPFull + 2,
               kOBarOFree = kOBarOFull + 1, kOBarRescReq = kOBarOFree + 1, kOBarRescDone = kOBarRescReq + 1,
               kOBarODrain = kOBarRescDone + 1, kOBarFin = kOBarODrain + 1, kONumBars = kOBarFin + 1;
 constexpr int kOOffTail = kOOffBar + kONumBars * 8;
-constexpr int kTailBytes = 32;  // tmem base, abort flag, resc slot, tile total
+constexpr int kTailBytes = 32;  // tmem base, abort flag, resc slot, tile total, first sequence and its tile
 constexpr int kSmemBytes = (kSOffTail > kOOffTail ? kSOffTail : kOOffTail) + kTailBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kSOffQR % 1024 == 0 && kSOffStage % 1024 == 0 && kOOffMsg % 1024 == 0 && kMsgStride % 1024 == 0,
@@ -136,21 +137,16 @@ struct Seg {
     int64_t blk0;  // first cache block of the sequence
 };
 
-// Walks the segments of one cluster's tile range [lo, hi).
+// Walks the segments of one cluster's tile range [lo, hi), starting at sequence b0 whose
+// first tile has global index tb0 (found once per CTA in the prologue).
 struct SegWalk {
     int b, tb, lo, hi, pidx;
-    __device__ void init(const Params& p, int lo_, int hi_, int pidx_) {
+    __device__ void init(int b0, int tb0, int lo_, int hi_, int pidx_) {
         lo = lo_;
         hi = hi_;
         pidx = pidx_;
-        b = 0;
-        tb = 0;
-        while (b < p.B) {
-            const int nt = seq_tiles(p, b);
-            if (tb + nt > lo) break;
-            tb += nt;
-            ++b;
-        }
+        b = b0;
+        tb = tb0;
     }
     __device__ bool next(const Params& p, Seg& s) {
         while (b < p.B && tb < hi) {
@@ -204,6 +200,7 @@ decode_tc_kernel(const Params p) {
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + tail + 4);
     volatile int* resc_pb = reinterpret_cast<volatile int*>(smem + tail + 8);
     int* nt_total = reinterpret_cast<int*>(smem + tail + 12);
+    int* walk0 = reinterpret_cast<int*>(smem + tail + 16);  // [first sequence of this cluster, its first tile]
     volatile int never = 0;  // abort flag for teardown waits (never raised)
 
     if ((sbase & 1023u) != 0) {  // identical in both CTAs: both leave here
@@ -241,6 +238,7 @@ decode_tc_kernel(const Params p) {
         fence_mbar_init();
     }
     if (warp == 0) {
+        // total tiles, then (by a warp scan) the sequence holding this cluster's first tile
         int s = 0;
         for (int b = lane; b < p.B; b += 32) {
             const int nt = seq_tiles(p, b);
@@ -254,7 +252,32 @@ decode_tc_kernel(const Params p) {
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) *nt_total = s;
+        const int pidx0 = static_cast<int>(blockIdx.x >> 1) % p.P_g;
+        const int lo0 = static_cast<int>((static_cast<int64_t>(pidx0) * s) / p.P_g);
+        int b0 = p.B, tb0 = s, run = 0;
+        for (int base = 0; base < p.B; base += 32) {
+            const int b = base + lane;
+            const int nt = b < p.B ? seq_tiles(p, b) : 0;
+            int inc = nt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            const unsigned hit = __ballot_sync(0xffffffffu, b < p.B && run + inc > lo0);
+            if (hit) {
+                const int f = __ffs(hit) - 1;
+                b0 = base + f;
+                tb0 = run + __shfl_sync(0xffffffffu, inc - nt, f);
+                break;
+            }
+            run += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) {
+            *nt_total = s;
+            walk0[0] = b0;
+            walk0[1] = tb0;
+        }
     }
     if (warp == kWarpProducer) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
@@ -268,6 +291,7 @@ decode_tc_kernel(const Params p) {
     const bool active = g < p.G;
     const int lo = static_cast<int>((static_cast<int64_t>(pidx) * Nt) / p.P_g);
     const int hi = static_cast<int>((static_cast<int64_t>(pidx + 1) * Nt) / p.P_g);
+    const int wb0 = walk0[0], wtb0 = walk0[1];
     const uint32_t peer_abort = mapa(sbase + (rank == 0 ? kOOffTail : kSOffTail) + 4, peer);
     const int64_t out_row_base = (static_cast<int64_t>(g) * p.slots) * kRows;
 
@@ -279,8 +303,8 @@ decode_tc_kernel(const Params p) {
             //      pulls whole blocks kPrefetchTiles ahead into L2.
             if (lane == 0) {
                 SegWalk w, wp;
-                w.init(p, lo, hi, pidx);
-                wp.init(p, lo, hi, pidx);
+                w.init(wb0, wtb0, lo, hi, pidx);
+                wp.init(wb0, wtb0, lo, hi, pidx);
                 Seg s, sp;
                 bool have_p = wp.next(p, sp);
                 int tp = have_p ? sp.t0 : 0;
@@ -323,7 +347,7 @@ decode_tc_kernel(const Params p) {
                 const uint64_t ring_desc = sdesc_sw128(sbase + kSOffRing, 16, 1024);
                 const uint64_t qr_desc = sdesc_sw128(sbase + kSOffQR, 16, 1024);
                 SegWalk w;
-                w.init(p, lo, hi, pidx);
+                w.init(wb0, wtb0, lo, hi, pidx);
                 Seg s;
                 uint32_t n = 0, kseg = 0, nc = 0;
                 bool ok = true;
@@ -381,7 +405,7 @@ decode_tc_kernel(const Params p) {
             const bool row_ok = rr < p.R;
             const int j = row_ok ? rr / p.H : 0;
             SegWalk w, wn;
-            w.init(p, lo, hi, pidx);
+            w.init(wb0, wtb0, lo, hi, pidx);
             Seg s, sn;
             uint32_t n = 0;
             bool failed = false;
@@ -506,7 +530,7 @@ decode_tc_kernel(const Params p) {
             const uint32_t peer_msg = mapa(sbase + kOOffMsg, peer);
             const uint32_t peer_pfull = mapa(sbase + kOOffBar + kOBarPFull * 8, peer);
             SegWalk w;
-            w.init(p, lo, hi, pidx);
+            w.init(wb0, wtb0, lo, hi, pidx);
             Seg s;
             uint32_t n = 0;
             bool failed = false;
@@ -544,7 +568,7 @@ decode_tc_kernel(const Params p) {
             //      as four bulk copies of 2 chunks into the ring of V stages
             if (lane == 0) {
                 SegWalk w;
-                w.init(p, lo, hi, pidx);
+                w.init(wb0, wtb0, lo, hi, pidx);
                 Seg s;
                 uint32_t nv = 0;  // stage loads issued
                 bool ok = true;
@@ -570,12 +594,12 @@ decode_tc_kernel(const Params p) {
         } else if (warp == kWarpMma) {
             // ---- MMA issuer (one thread): O += P V (A = P, K-major SW128; B = V, MN-major SW128
             //      with 16 KB between 64-column atoms)
-            constexpr uint32_t idesc = idesc_bf16_f32(kRows, 128, false, true);
+            constexpr uint32_t idesc = idesc_bf16_f32(kRows, 64 * kVChunksPerStage, false, true);
             const uint32_t peer_pempty = mapa(sbase + kSOffBar + kSBarPEmpty * 8, peer);
             const uint64_t p_desc = sdesc_sw128(sbase + kOOffMsg, 16, 1024);
             const uint64_t v_desc = sdesc_sw128(sbase + kOOffV, kChunk, 1024);
             SegWalk w;
-            w.init(p, lo, hi, pidx);
+            w.init(wb0, wtb0, lo, hi, pidx);
             Seg s;
             uint32_t n = 0, nv = 0, kseg = 0, nresc = 0;
             bool ok = true;
@@ -631,7 +655,7 @@ decode_tc_kernel(const Params p) {
                             const uint64_t pd = p_desc + (static_cast<uint64_t>(pb * kMsgStride) >> 4);
 #pragma unroll
                             for (int kk = 0; kk < kTile / 16; ++kk)
-                                mma_ss(tmem + 128 * k, pd + (((kk >> 2) * kRows * 128 + (kk & 3) * 32) >> 4),
+                                mma_ss(tmem + 64 * kVChunksPerStage * k, pd + (((kk >> 2) * kRows * 128 + (kk & 3) * 32) >> 4),
                                        vd + ((kk * 2048) >> 4), idesc, (first && kk == 0) ? 0u : 1u);
                             mma_commit(smem_u32(&bars[kOBarVEmpty + st]));
                         }
@@ -659,7 +683,7 @@ decode_tc_kernel(const Params p) {
             const int rr = g * kRows + r;
             const bool row_ok = rr < p.R;
             SegWalk w;
-            w.init(p, lo, hi, pidx);
+            w.init(wb0, wtb0, lo, hi, pidx);
             Seg s;
             uint32_t kseg = 0, nresc = 0;
             bool ok = true;
