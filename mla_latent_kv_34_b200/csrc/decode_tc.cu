@@ -89,7 +89,8 @@ constexpr int kSOffRing = 0;                                  // 4 x 48 KB
 constexpr int kSOffQR = kRingSlots * kCopyBytes;              // RoPE part of Q: [128 x 64] swizzled, 16 KB
 constexpr int kSOffStage = kSOffQR + kRows * 128;             // the P message being built (kMsgBytes)
 constexpr int kSOffXchg = kSOffStage + kMsgStride;            // [2][128] fp32 half-row maxima / sums
-constexpr int kSOffBar = kSOffXchg + 2 * kRows * 4;
+constexpr int kSOffQT = kSOffXchg + 2 * kRows * 4;            // 8 warps x [32 rows x 128 B] Q transpose tiles
+constexpr int kSOffBar = kSOffQT + kSoftWarps * 32 * 128;
 constexpr int kSBarFull = 0, kSBarEmpty = kRingSlots, kSBarSFull = 2 * kRingSlots, kSBarSEmpty = kSBarSFull + 2,
               kSBarPEmpty = kSBarSEmpty + 2, kSBarQReady = kSBarPEmpty + 2, kSBarFin = kSBarQReady + 1,
               kSNumBars = kSBarFin + 1;
@@ -115,7 +116,7 @@ struct Params {
     const uint8_t* cache;  // blocks of kBlockBytes
     const int64_t* seq_block;
     const int32_t* kv_len;
-    float* o_part;    // [G][slots][128][512]
+    float* o_part;    // [G][slots][128 column groups of 4][128 rows] x float4 (unnormalised O)
     float2* ml_part;  // [G][slots][128]  (running max in log2 units, sum)
     int32_t* dev_status;
     int64_t cap_blocks;
@@ -413,35 +414,61 @@ decode_tc_kernel(const Params p) {
             while (!failed && have) {
                 wn = w;
                 const bool have_next = wn.next(p, sn);
-                // this segment's absorbed query row: latent part -> TMEM columns 0..255 (warp
-                // hf=0: columns 0..127, hf=1: 128..255), RoPE part -> shared memory row r
-                // (hf=0: units 0..3, hf=1: units 4..7).  The next segment's row goes to L2.
-                const uint16_t* qrow = p.q + (static_cast<int64_t>(s.b) * p.R + (row_ok ? rr : 0)) * kRow;
-                if (have_next && row_ok) {
-                    const char* nq = reinterpret_cast<const char*>(p.q + (static_cast<int64_t>(sn.b) * p.R + rr) * kRow);
-                    for (int c = hf; c < 9; c += 2) prefetch_l2(nq + 128 * c);
-                }
+                // this segment's absorbed query rows: latent part -> TMEM columns 0..255 (warp
+                // hf=0: columns 0..127, hf=1: 128..255), RoPE part -> shared memory (hf=0: units
+                // 0..3, hf=1: units 4..7).  The warp loads its 32 rows coalesced (a lane per
+                // 16-byte unit) and transposes each 64-column chunk through a swizzled 4 KB tile
+                // into the lane-per-row order of tcgen05.st.  The next segment's rows are pulled
+                // into L2 two tiles before this segment ends (earlier, the streamed cache would
+                // evict them).
+                const int64_t qrow0 = static_cast<int64_t>(s.b) * p.R + g * kRows + 32 * qd;
+                const int t_pf = max(s.t0, s.t1 - 2);
+                const char* nq = (have_next && row_ok) ? reinterpret_cast<const char*>(
+                                                              p.q + (static_cast<int64_t>(sn.b) * p.R + rr) * kRow)
+                                                        : nullptr;
                 __syncwarp();
                 {
-                    const uint4* src = reinterpret_cast<const uint4*>(qrow);
+                    uint8_t* qt = smem + kSOffQT + warp * (32 * 128);
+                    const int lu = lane & 7, lr = lane >> 3;  // unit and row-in-quad of this lane's loads
 #pragma unroll 1
                     for (int c = 4 * hf; c < 4 * hf + 4; c += 2) {
-                        uint32_t v0[32], v1[32];
+                        uint4 x[2][8];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const uint4 x = row_ok ? src[8 * c + k] : make_uint4(0, 0, 0, 0);
-                            const uint4 y = row_ok ? src[8 * c + 8 + k] : make_uint4(0, 0, 0, 0);
-                            v0[4 * k] = x.x; v0[4 * k + 1] = x.y; v0[4 * k + 2] = x.z; v0[4 * k + 3] = x.w;
-                            v1[4 * k] = y.x; v1[4 * k + 1] = y.y; v1[4 * k + 2] = y.z; v1[4 * k + 3] = y.w;
+                        for (int j = 0; j < 2; ++j)
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int ri = 4 * i + lr;
+                                x[j][i] = make_uint4(0, 0, 0, 0);
+                                if (g * kRows + 32 * qd + ri < p.R)
+                                    x[j][i] = reinterpret_cast<const uint4*>(p.q + (qrow0 + ri) * kRow)[8 * (c + j) + lu];
+                            }
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int ri = 4 * i + lr;
+                                *reinterpret_cast<uint4*>(qt + ri * 128 + ((lu ^ (ri & 7)) << 4)) = x[j][i];
+                            }
+                            __syncwarp();
+                            uint32_t v[32];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const uint4 y = *reinterpret_cast<const uint4*>(qt + lane * 128 + ((u ^ (lane & 7)) << 4));
+                                v[4 * u] = y.x; v[4 * u + 1] = y.y; v[4 * u + 2] = y.z; v[4 * u + 3] = y.w;
+                            }
+                            __syncwarp();
+                            tmem_st32(t_lane + kColQ + 32 * (c + j), v);
                         }
-                        tmem_st32(t_lane + kColQ + 32 * c, v0);
-                        tmem_st32(t_lane + kColQ + 32 * (c + 1), v1);
                     }
-                    uint8_t* qr = smem + kSOffQR + r * 128;
+                    // RoPE part: rows 8 i + lane / 4, unit 4 hf + lane % 4, straight into its swizzled rows
 #pragma unroll
-                    for (int u = 4 * hf; u < 4 * hf + 4; ++u) {
-                        const uint4 x = row_ok ? src[64 + u] : make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4*>(qr + ((u ^ (r & 7)) << 4)) = x;
+                    for (int i = 0; i < 4; ++i) {
+                        const int ri = 8 * i + (lane >> 2), u = 4 * hf + (lane & 3);
+                        uint4 y = make_uint4(0, 0, 0, 0);
+                        if (g * kRows + 32 * qd + ri < p.R)
+                            y = reinterpret_cast<const uint4*>(p.q + (qrow0 + ri) * kRow)[64 + u];
+                        const int R = 32 * qd + ri;
+                        *reinterpret_cast<uint4*>(smem + kSOffQR + R * 128 + ((u ^ (R & 7)) << 4)) = y;
                     }
                 }
                 fence_proxy_async_cta();
@@ -452,6 +479,8 @@ decode_tc_kernel(const Params p) {
                 float m = -CUDART_INF_F, l = 0.f;
                 for (int t = s.t0; t < s.t1; ++t, ++n) {
                     const uint32_t sb = n & 1u, us = n >> 1;
+                    if (t == t_pf && have_next && row_ok)
+                        for (int c = hf; c < 9; c += 2) prefetch_l2(nq + 128 * c);
                     bool ok = mbar_wait(&bars[kSBarSFull + sb], us & 1u, abort_flag, kLimitNs);
                     __syncwarp();
                     tc_fence_after();
@@ -743,19 +772,21 @@ decode_tc_kernel(const Params p) {
                 __syncwarp();
                 if (!ok) break;
                 tc_fence_after();
-                float* orow = p.o_part + (out_row_base + static_cast<int64_t>(s.slot) * kRows + r) * kDc;
+                // column group j (4 latent columns) of all 128 rows is contiguous, so each warp store
+                // below writes 512 consecutive bytes (row-per-thread stores of row-major O would
+                // scatter every warp store over 32 rows)
+                float4* oseg = reinterpret_cast<float4*>(p.o_part) +
+                               (out_row_base + static_cast<int64_t>(s.slot) * kRows) * (kDc / 4);
 #pragma unroll 1
                 for (int c = 0; c < 16; ++c) {
                     uint32_t v[32];
                     tmem_ld32(t_lane + 32 * c, v);
                     tmem_wait_ld();
-                    if (row_ok) {
-                        float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            dst[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                                                 __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
-                    }
+                    for (int k = 0; k < 8; ++k)
+                        oseg[(8 * c + k) * kRows + r] =
+                            make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                                        __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
                 }
                 tc_fence_before();
                 mbar_arrive(&bars[kOBarOFree]);

@@ -334,10 +334,11 @@ __global__ void __launch_bounds__(kFinThreads, 1) finish_tc_kernel(
                             wi[u] = __shfl_sync(0xffffffffu, w, (i0 + u) & 31);
                             if (i0 + u >= cnt) wi[u] = 0.f;
                             if (wi[u] != 0.f) {
-                                const float4* src = reinterpret_cast<const float4*>(
-                                    o_part + ((seg0 + base + i0 + u) * 128 + row) * kDc + 16 * lane);
+                                // segment partials: [column group of 4][128 rows] x float4
+                                const float4* src = reinterpret_cast<const float4*>(o_part) +
+                                                    ((seg0 + base + i0 + u) * 128 + 4 * lane) * 128 + row;
 #pragma unroll
-                                for (int k = 0; k < 4; ++k) v[u][k] = src[k];
+                                for (int k = 0; k < 4; ++k) v[u][k] = src[k * 128];
                             }
                         }
 #pragma unroll

@@ -145,6 +145,13 @@ __device__ __forceinline__ void bulk_load(uint32_t smem_dst, const void* src, ui
                  : "memory");
 }
 
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to global memory, tracked
+// by the bulk async-group of the issuing thread (commit, then wait_group / wait_group.read).
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t smem_src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_src), "r"(bytes)
+                 : "memory");
+}
+
 // Pull `bytes` of global memory into L2 (no shared memory, no barrier).
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
@@ -190,6 +197,11 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
         : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups are still in flight.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
 // Wait until at most N committed bulk groups still read their source.
 template <int N>
 __device__ __forceinline__ void bulk_wait_group_read() {
