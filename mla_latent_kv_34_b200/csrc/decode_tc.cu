@@ -63,7 +63,6 @@ constexpr int kVChunksPerStage = 4;  // O CTA: a V stage = 4 chunks (64 KB) = on
 constexpr int kVStageBytes = kVChunksPerStage * kChunk;
 constexpr int kVPerTile = 8 / kVChunksPerStage;  // V stages per tile (the 8 latent chunks)
 constexpr int kVStages = 2;          // O CTA: ring of V stages
-constexpr int kPrefetchTiles = 1;    // S CTA: blocks pulled into L2 ahead of the ring
 constexpr int kPBytes = kRows * kTile * 2;       // 32 KB bf16 P tile: two [128 x 64] swizzled atoms
 constexpr int kMsgBytes = kPBytes + kRows * 4;  // P | alpha[128] (per-row rescale factors): one bulk copy
 constexpr int kMsgStride = 33792;    // 1024-aligned message slots in the O CTA
@@ -300,37 +299,26 @@ decode_tc_kernel(const Params p) {
         // =============================================================== S CTA
         if (warp == kWarpProducer) {
             // ---- copy producer: each 128-token block (144 KB, already in the operand layout)
-            //      lands as three 48 KB bulk copies, one per ring slot.  A second walker
-            //      pulls whole blocks kPrefetchTiles ahead into L2.
+            //      lands as three 48 KB bulk copies, one per ring slot, marked to stay in L2
+            //      for the O CTA's read of the latent part.  (Pulling blocks into L2 ahead of
+            //      the ring was measured to lose them to eviction and only add DRAM reads.)
             if (lane == 0) {
-                SegWalk w, wp;
+                SegWalk w;
                 w.init(wb0, wtb0, lo, hi, pidx);
-                wp.init(wb0, wtb0, lo, hi, pidx);
-                Seg s, sp;
-                bool have_p = wp.next(p, sp);
-                int tp = have_p ? sp.t0 : 0;
-                auto prefetch_one = [&]() {
-                    if (!have_p) return;
-                    bulk_prefetch_l2(p.cache + (sp.blk0 + tp) * kBlockBytes, kBlockBytes);
-                    if (++tp >= sp.t1) {
-                        have_p = wp.next(p, sp);
-                        tp = have_p ? sp.t0 : 0;
-                    }
-                };
-                for (int i = 0; i < kPrefetchTiles; ++i) prefetch_one();
+                Seg s;
                 uint32_t nc = 0;  // copies issued
                 bool ok = true;
+                const uint64_t keep = l2_policy_evict_last();
                 while (ok && w.next(p, s)) {
                     for (int t = s.t0; ok && t < s.t1; ++t) {
-                        prefetch_one();
                         const uint8_t* src = p.cache + (s.blk0 + t) * kBlockBytes;
                         for (int k = 0; k < kCopies; ++k, ++nc) {
                             const uint32_t slot = nc % kRingSlots, u = nc / kRingSlots;
                             ok = mbar_wait(&bars[kSBarEmpty + slot], (u & 1u) ^ 1u, abort_flag, kLimitNs);
                             if (!ok) break;
                             mbar_arrive_expect_tx(&bars[kSBarFull + slot], kCopyBytes);
-                            bulk_load(sbase + kSOffRing + slot * kCopyBytes, src + k * kCopyBytes, kCopyBytes,
-                                      &bars[kSBarFull + slot]);
+                            bulk_load_hint(sbase + kSOffRing + slot * kCopyBytes, src + k * kCopyBytes, kCopyBytes,
+                                           &bars[kSBarFull + slot], keep);
                         }
                     }
                 }
@@ -601,6 +589,7 @@ decode_tc_kernel(const Params p) {
                 Seg s;
                 uint32_t nv = 0;  // stage loads issued
                 bool ok = true;
+                const uint64_t last_use = l2_policy_evict_first();
                 while (ok && w.next(p, s)) {
                     for (int t = s.t0; ok && t < s.t1; ++t) {
                         const uint8_t* src = p.cache + (s.blk0 + t) * kBlockBytes;
@@ -611,8 +600,8 @@ decode_tc_kernel(const Params p) {
                                 break;
                             }
                             mbar_arrive_expect_tx(&bars[kOBarVFull + st], kVStageBytes);
-                            bulk_load(sbase + kOOffV + st * kVStageBytes, src + k * kVStageBytes, kVStageBytes,
-                                      &bars[kOBarVFull + st]);
+                            bulk_load_hint(sbase + kOOffV + st * kVStageBytes, src + k * kVStageBytes, kVStageBytes,
+                                           &bars[kOBarVFull + st], last_use);
                         }
                     }
                 }
