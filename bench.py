@@ -48,7 +48,9 @@ CORE_SOURCES = ["mla_latent_kv_34_b200/csrc/decode_tc.cu", "mla_latent_kv_34_b20
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 3000 for the CUDA path: about a second, so the clock sampler sees "
+                         "the timed region; 20 oracle samples for --impl reference)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="v2", choices=sorted(mi.CONFIGS))
@@ -125,7 +127,8 @@ class ClockSampler:
         self.proc = None
         self.path = None
 
-    def start(self):
+    def start(self, skip: int = 3):
+        self.skip = skip
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "100"]
@@ -155,6 +158,7 @@ class ClockSampler:
             except ValueError:
                 continue
         os.unlink(self.path)
+        rows = rows[self.skip:]  # samples taken while the sampler was settling, before the timed region
         if not rows:
             return None
         reasons = set()
@@ -509,6 +513,8 @@ def run_reference(args, dist):
 
 def main():
     args = parse_args()
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" else 3000
     dist = Dist(args.gpus)
     if args.impl == "reference":
         run_reference(args, dist)
