@@ -174,32 +174,45 @@ class ClockSampler:
 # ------------------------------------------------------------------ distributed plumbing
 
 class Dist:
-    def __init__(self, gpus: int):
+    """One process per GPU (torchrun env vars); NCCL for the barrier and the max / sum reductions.
+
+    backend="gloo" runs the same plumbing on CPU ranks (used by the multi-process tests).
+    """
+
+    def __init__(self, gpus: int, backend: str = "nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
         self.pg = False
         if gpus > 1 and self.world != gpus:
             raise SystemExit(f"--gpus {gpus} needs torchrun with {gpus} processes (WORLD_SIZE={self.world})")
 
+    def _device(self, torch):
+        return torch.device("cuda", self.local_rank) if self.backend == "nccl" else torch.device("cpu")
+
     def init(self, torch):
-        torch.cuda.set_device(self.local_rank)
+        if self.backend == "nccl":
+            torch.cuda.set_device(self.local_rank)
         if self.world > 1:
             import torch.distributed as dist
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local_rank))
+            kw = {"device_id": self._device(torch)} if self.backend == "nccl" else {}
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120), **kw)
             self.pg = True
 
     def barrier(self, torch):
         if self.pg:
             import torch.distributed as dist
-            dist.barrier(device_ids=[self.local_rank])
+            if self.backend == "nccl":
+                dist.barrier(device_ids=[self.local_rank])
+            else:
+                dist.barrier()
 
     def reduce(self, torch, value: float, op: str) -> float:
         if not self.pg:
             return value
         import torch.distributed as dist
-        t = torch.tensor([value], dtype=torch.float64, device="cuda")
+        t = torch.tensor([value], dtype=torch.float64, device=self._device(torch))
         dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
         return float(t.item())
 
@@ -207,6 +220,20 @@ class Dist:
         if self.pg:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+def rank_config(base: mi.MLAConfig, rank: int) -> mi.MLAConfig:
+    """Each rank decodes its own batch of the same shape (weak scaling): only the seed differs."""
+    return mi.MLAConfig(**{**base.__dict__, "seed": base.seed + 7919 * rank})
+
+
+def aggregate(dist, torch, step_ms: list, step_bytes: float) -> tuple:
+    """Weak scaling: each rank times its own batch; the job's time per step is the slowest rank's,
+    its work the sum over ranks.  Returns (ms_per_step, TB/s of the whole job)."""
+    total_ms = dist.reduce(torch, sum(step_ms), "max")
+    ms_per_step = total_ms / len(step_ms)
+    bytes_all = dist.reduce(torch, float(step_bytes), "sum")
+    return ms_per_step, bytes_all / (ms_per_step * 1e-3) / 1e12
 
 
 # ------------------------------------------------------------------ our arm
@@ -303,7 +330,7 @@ def run_ours(args, dist):
     import mla_latent_kv_34_b200 as mla
     dev = torch.device("cuda", dist.local_rank)
     base = mi.CONFIGS[args.config]
-    cfg = mi.MLAConfig(**{**base.__dict__, "seed": base.seed + 7919 * dist.rank})
+    cfg = rank_config(base, dist.rank)
     st = build_state(torch, mla, cfg, dev)
     counts = step_counts(cfg, st["lengths"])
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -360,12 +387,10 @@ def run_ours(args, dist):
     if int(st["status"].item()) != 0:
         raise SystemExit(f"device status {mla.device_status_string(int(st['status'].item()))}")
     del g_step, g_parts
-    total_ms = dist.reduce(torch, sum(step_ms), "max")
     core_mean_ms = dist.reduce(torch, statistics.mean(core_ms), "max")
-    ms_per_step = total_ms / args.steps
+    ms_per_step, value = aggregate(dist, torch, step_ms, counts["step_bytes"])
     bytes_all = dist.reduce(torch, float(counts["step_bytes"]), "sum")
     flops_all = dist.reduce(torch, float(counts["step_flops"]), "sum")
-    value = bytes_all / (ms_per_step * 1e-3) / 1e12
 
     # end-to-end through the public API with host buffers
     e2e = None

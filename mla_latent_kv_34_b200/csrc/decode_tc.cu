@@ -698,8 +698,6 @@ decode_tc_kernel(const Params p) {
             // ---- epilogue: warps 0..3, one thread per query row
             const int r = tid;
             const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-            const int rr = g * kRows + r;
-            const bool row_ok = rr < p.R;
             SegWalk w;
             w.init(wb0, wtb0, lo, hi, pidx);
             Seg s;
