@@ -11,8 +11,8 @@
 //     (the A operand, 256 columns of packed bf16 pairs), the RoPE part in shared
 //     memory.  Each 128-token cache block (9 pre-swizzled [128 x 64] chunks,
 //     144 KB) arrives as three 48 KB bulk copies into a ring of three copy slots
-//     (blocks are pulled into L2 several tiles ahead, so the ring's copies hit
-//     L2), and S = Q K^T is formed by 36 tcgen05.mma (M=128, N=128, K=16:
+//     (marked evict_last in L2, so that CTA 1's read of the same block hits L2),
+//     and S = Q K^T is formed by 36 tcgen05.mma (M=128, N=128, K=16:
 //     full-rate shape) into one of two TMEM score buffers.  Eight warps (a query
 //     row's 128 scores split over two threads) run the online softmax in fp32
 //     and stage P (bf16) in shared memory; a sender warp ships each staged P

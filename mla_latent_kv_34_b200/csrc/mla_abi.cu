@@ -34,7 +34,8 @@ DecodeWs decode_ws_layout(int B, int n_q, int H, int S) {
 
 mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
-// ---- tensor-core path: segment partials [G][slots][128] x (float2 ml, 512 fp32 O)
+// ---- tensor-core path: segment partials [G][slots][128 rows] float2 (m, l), then (1024-aligned)
+//      [G][slots] blocks of 128 rows x 512 fp32 O, each stored as [128 column groups of 4][128 rows] x float4
 struct TcWs {
     int G, slots;
     size_t ml_part, o_part, total;

@@ -10,9 +10,9 @@
 //           W^UV is applied after the aggregation in latent space ("两张账" page).
 //
 // One CTA per (head, block of up to 64 query rows t).  The head's weight matrix
-// [128 x 512] bf16 lands in shared memory with one TMA box through a 3-D view
-// (column within a 64-column chunk, row, chunk), giving eight [128 x 64] chunks
-// with the 128-byte swizzle.  The token-side operand is staged by the CTA's
+// [128 x 512] bf16 lands in shared memory as eight TMA boxes through a 3-D view
+// (column within a 64-column chunk, row, chunk), one [128 x 64] chunk each, with
+// the 128-byte swizzle.  The token-side operand is staged by the CTA's
 // threads into the same swizzled layout; one thread issues the MMAs (M = 128,
 // N = token block, K = 16) with the accumulator in TMEM; four warps read it back.
 #include <cuda.h>
