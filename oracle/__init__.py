@@ -22,7 +22,8 @@ Sources (the pages describing DeepSeek-V2 Multi-head Latent Attention):
 Modules:
   naive   -- fp64 naive decode (explicit k^C, v^C per head; textbook softmax),
              the fp64 absorbed form, split-KV partials and their LSE merge,
-             RoPE, cache-footprint formulas.
+             RoPE, cache-footprint formulas, and the query-side up-projections
+             q^C = W^UQ c^Q, q^R = W^QR c^Q of the compressed query.
   append  -- bit-exact emulation of the cache append in the kernel's fp32
              arithmetic (RoPE table rounded to fp32; separate multiplies and
              adds; round-to-nearest-even to bf16).
@@ -32,4 +33,6 @@ Readings taken where the pages are silent (each is a documented choice):
   * RoPE pairs adjacent dims (2i, 2i+1), theta_i = base^(-2i/d_h^R), base 10000;
   * the key at cache index t has position t; query j of a step with n_q new
     tokens has position L_b - n_q + j and sees keys t <= L_b - n_q + j.
+  * q^R is an up-projection of the compressed query c^Q, like q^C (its formula
+    is lost on the pages).
 """

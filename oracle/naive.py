@@ -210,3 +210,23 @@ def up_project(o_lat: np.ndarray, W_UV: np.ndarray) -> np.ndarray:
 def absorb_query(q_nope: np.ndarray, W_UK: np.ndarray) -> np.ndarray:
     """q_abs[t, h] = (W^UK_h)^T q_nope[t, h]  ([T, H, 128] -> [T, H, 512])."""
     return np.einsum("hdc,thd->thc", _f64(W_UK), _f64(q_nope))
+
+
+# --------------------------------------------------------------------------
+# Query side of the low-rank path (explainer 2.2.1.2: queries are compressed
+# like K/V, a down-projection to c^Q then up-projections; q^C_t = W^UQ c^Q_t;
+# 2.2.2: the decoupled per-head q^R)
+# --------------------------------------------------------------------------
+
+def query_up(c_q: np.ndarray, W_UQ: np.ndarray, W_QR: np.ndarray):
+    """q^C[t, h] = W^UQ_h c^Q_t (128) and q^R[t, h] = W^QR_h c^Q_t (64, not yet rotated).
+
+    c_q [T, d_c'], W_UQ [H, 128, d_c'], W_QR [H, 64, d_c'] -> ([T, H, 128], [T, H, 64]).
+    Reading: both query parts come from the compressed query c^Q (the pages print
+    q^C = W^UQ c^Q; the formula for q^R is lost, and "compressed the same way as
+    K/V" is read as q^R also being an up-projection of c^Q).  The rotation R_p of
+    q^R happens in the absorb step, at the query's position.
+    """
+    c_q = _f64(c_q)
+    return (np.einsum("hdk,tk->thd", _f64(W_UQ), c_q),
+            np.einsum("hdk,tk->thd", _f64(W_QR), c_q))

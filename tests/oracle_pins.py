@@ -195,3 +195,56 @@ def check_absorbed_identity(attend, absorbed) -> None:
 ALL_SINGLE = (check_single_token, check_constant_values, check_zero_query,
               check_scale_closed_form, check_rope_closed_form,
               check_causal_within_pair, check_brute_force)
+
+
+# ---------------------------------------------------------------- query side (q^C, q^R from c^Q)
+
+def query_weights(H: int, d_cq: int, seed: int):
+    """Random W^UQ [H,128,d_cq], W^QR [H,64,d_cq] with variance 1/d_cq, and c^Q ~ N(0,1) rows."""
+    g = lambda s, n, sig=1.0: bf16_bits_to_f64(normal_bf16(seed, s, 0, n, sig))
+    Wuq = g(21, H * D_H * d_cq, 1 / math.sqrt(d_cq)).reshape(H, D_H, d_cq)
+    Wqr = g(22, H * D_R * d_cq, 1 / math.sqrt(d_cq)).reshape(H, D_R, d_cq)
+    return Wuq, Wqr
+
+
+def check_query_up_selection(query_up) -> None:
+    """Selection weights give slices of c^Q in closed form.
+
+    Head h's W^UQ_h picks columns (7h + d + 1) mod d_c' (d = 0..127) and W^QR_h
+    picks columns (5h + 2i + 3) mod d_c' (i = 0..63): one 1 per row, so
+    q^C[t, h, d] = c^Q[t, (7h + d + 1) mod d_c'] and likewise for q^R.  A
+    transposed weight, a head read from another head's weights, or the two
+    projections swapped all give different slices.
+    """
+    T, H, d_cq = 3, 4, 320
+    rng = np.random.default_rng(17)
+    cq = rng.standard_normal((T, d_cq))
+    Wuq = np.zeros((H, D_H, d_cq))
+    Wqr = np.zeros((H, D_R, d_cq))
+    for h in range(H):
+        Wuq[h, np.arange(D_H), (7 * h + np.arange(D_H) + 1) % d_cq] = 1.0
+        Wqr[h, np.arange(D_R), (5 * h + 2 * np.arange(D_R) + 3) % d_cq] = 1.0
+    qn, qr = query_up(cq, Wuq, Wqr)
+    assert qn.shape == (T, H, D_H) and qr.shape == (T, H, D_R)
+    for h in range(H):
+        np.testing.assert_array_equal(qn[:, h], cq[:, (7 * h + np.arange(D_H) + 1) % d_cq])
+        np.testing.assert_array_equal(qr[:, h], cq[:, (5 * h + 2 * np.arange(D_R) + 3) % d_cq])
+
+
+def check_query_absorb_precomposed(query_up, absorb_query) -> None:
+    """Query path then absorption equals the precomposed matrix (W^UK_h)^T W^UQ_h applied to c^Q.
+
+    The precomposed product is formed here with one matmul per head, a different
+    order of the same sums, so a dropped head, a wrong contraction axis or a
+    transposed factor shows as a mismatch far above fp64 rounding.
+    """
+    T, H, d_cq = 5, 3, 192
+    Wuq, Wqr = query_weights(H, d_cq, 31)
+    _, _, _, _, Wk, _ = rand_problem(1, H, 1, 32)
+    cq = bf16_bits_to_f64(normal_bf16(33, 1, 0, T * d_cq)).reshape(T, d_cq)
+    qn, qr = query_up(cq, Wuq, Wqr)
+    q_abs = absorb_query(qn, Wk)
+    for h in range(H):
+        M = Wk[h].T @ Wuq[h]                                   # [512, d_cq]
+        np.testing.assert_allclose(q_abs[:, h], cq @ M.T, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(qr[:, h], cq @ Wqr[h].T, rtol=1e-12, atol=1e-13)

@@ -90,3 +90,51 @@ def test_pins_reject_planted_mistake(name, monkeypatch):
             caught.append(check.__name__)
             break
     assert caught, f"no pin caught mutation {name}"
+
+
+# ---------------------------------------------------------------- query side
+
+def _qup_transposed(cq, Wuq, Wqr):
+    # the square leading block of each head's W^UQ used transposed
+    W2 = Wuq.copy()
+    W2[:, :, :128] = np.swapaxes(Wuq[:, :, :128], 1, 2)
+    return on.query_up(cq, W2, Wqr)
+
+
+def _qup_head_shift(cq, Wuq, Wqr):
+    # head h reads head h+1's weights
+    return on.query_up(cq, np.roll(Wuq, -1, axis=0), np.roll(Wqr, -1, axis=0))
+
+
+def _qup_rope_from_content(cq, Wuq, Wqr):
+    # q^R taken from the first 64 rows of W^UQ instead of W^QR
+    return on.query_up(cq, Wuq, Wuq[:, :64])
+
+
+def _qup_dropped_column(cq, Wuq, Wqr):
+    # the last column of c^Q left out of the contraction
+    cq2 = np.array(cq, dtype=np.float64)
+    cq2[:, -1] = 0.0
+    return on.query_up(cq2, Wuq, Wqr)
+
+
+QUERY_MUTATIONS = {
+    "w_uq_index_transposed": _qup_transposed,
+    "query_head_shifted": _qup_head_shift,
+    "q_rope_from_w_uq": _qup_rope_from_content,
+    "c_q_last_column_dropped": _qup_dropped_column,
+}
+
+
+@pytest.mark.parametrize("name", sorted(QUERY_MUTATIONS))
+def test_query_pins_reject_planted_mistake(name):
+    mutated = QUERY_MUTATIONS[name]
+    caught = False
+    for check in (pins.check_query_up_selection,
+                  lambda f: pins.check_query_absorb_precomposed(f, on.absorb_query)):
+        try:
+            check(mutated)
+        except AssertionError:
+            caught = True
+            break
+    assert caught, f"no query-side pin caught mutation {name}"

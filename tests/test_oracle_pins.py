@@ -141,3 +141,11 @@ def test_rope_table_matches_closed_values():
     assert np.all(c[0] == 1.0) and np.all(s[0] == 0.0)
     assert c[1, 0] == np.float32(math.cos(1.0)) and s[1, 0] == np.float32(math.sin(1.0))
     assert s[2, 16] == np.float32(math.sin(100 * 0.01))
+
+
+def test_query_up_selection_closed_form():
+    pins.check_query_up_selection(on.query_up)
+
+
+def test_query_up_then_absorb_equals_precomposed():
+    pins.check_query_absorb_precomposed(on.query_up, on.absorb_query)
