@@ -108,6 +108,32 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* p
                         int T, int H, void* q_out, int32_t* dev_status, mla_stream stream);
 
 /*
+ * mla_query_up -- the query side of the low-rank path: up-projections of the
+ * compressed query c^Q into the content query q^C and the RoPE query q^R.
+ * (MLA explainer 2.2.1.2: queries are compressed like keys and values, a
+ *  down-projection to c^Q and up-projections from it, q^C_t = W^UQ c^Q_t;
+ *  2.2.2: the decoupled per-head q^R.  q^R = W^QR c^Q is this library's
+ *  reading: its formula is lost on the page.)
+ *   c_q     bf16 [T, d_cq]        compressed queries c^Q (row-major)
+ *   W_UQ    bf16 [H, 128, d_cq]   per-head content up-projection
+ *   W_QR    bf16 [H, 64, d_cq]    per-head RoPE up-projection
+ *   q_nope  bf16 [T, H, 128]      out: q^C[t, h] = W^UQ_h c^Q_t
+ *   q_rope  bf16 [T, H, 64]       out: q^R[t, h] = W^QR_h c^Q_t, not rotated
+ *                                 (mla_absorb_q rotates it at the query position)
+ * The outputs are exactly mla_absorb_q's inputs.  fp32 accumulation on the
+ * tensor cores, one rounding to bf16 per output element.
+ * Sizes: 1 <= H <= 128; d_cq a multiple of 64 in [64, 16384]; T >= 0 (T = 0
+ * launches nothing).  All pointers are device memory owned by the caller,
+ * 16-byte aligned; nothing is kept after the call returns.
+ * Errors: MLA_ERR_UNSUPPORTED_SHAPE for H or d_cq out of range,
+ * MLA_ERR_INVALID_ARG for null or misaligned pointers or T < 0 (returned
+ * before any launch); MLA_ERR_CUDA if the launch fails; an expired bounded
+ * wait on the device sets MLA_DEVERR_TIMEOUT in *dev_status (may be NULL).
+ */
+mla_status mla_query_up(const void* c_q, const void* W_UQ, const void* W_QR, int T, int H, int d_cq,
+                        void* q_nope, void* q_rope, int32_t* dev_status, mla_stream stream);
+
+/*
  * mla_append_cache -- write T new tokens into the blocked latent cache.
  * ("两张账" page: only c^KV and k^R are cached; explainer 2.2.2: k^R is
  *  cached already rotated.)

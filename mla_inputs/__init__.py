@@ -47,6 +47,9 @@ STREAM_Q_ROPE = 4
 STREAM_W_UK = 5
 STREAM_W_UV = 6
 STREAM_LENGTHS = 7
+STREAM_C_Q = 8
+STREAM_W_UQ = 9
+STREAM_W_QR = 10
 
 
 def _mix64(z: np.ndarray) -> np.ndarray:
@@ -216,6 +219,16 @@ def weights(cfg: MLAConfig, which: str) -> np.ndarray:
     stream = {"uk": STREAM_W_UK, "uv": STREAM_W_UV}[which]
     n = cfg.H * D_H * D_C
     return normal_bf16(cfg.seed, stream, 0, n, 1.0 / np.sqrt(D_C)).reshape(cfg.H, D_H, D_C)
+
+
+def compressed_queries(cfg: MLAConfig, d_cq: int):
+    """Compressed queries and their up-projections, bf16 bits: c^Q [T, d_cq] ~ N(0, 1),
+    W^UQ [H, 128, d_cq] and W^QR [H, 64, d_cq] ~ N(0, 1/d_cq) (so q^C and q^R are ~N(0, 1))."""
+    cq = normal_bf16(cfg.seed, STREAM_C_Q, 0, cfg.T * d_cq).reshape(cfg.T, d_cq)
+    sig = 1.0 / np.sqrt(d_cq)
+    wuq = normal_bf16(cfg.seed, STREAM_W_UQ, 0, cfg.H * D_H * d_cq, sig).reshape(cfg.H, D_H, d_cq)
+    wqr = normal_bf16(cfg.seed, STREAM_W_QR, 0, cfg.H * D_R * d_cq, sig).reshape(cfg.H, D_R, d_cq)
+    return cq, wuq, wqr
 
 
 def token_rows(cfg: MLAConfig, row0: int, nrows: int):

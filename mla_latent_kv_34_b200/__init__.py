@@ -34,6 +34,7 @@ _SIGS = {
     "mla_device_status_string": ([ctypes.c_int32], ctypes.c_char_p),
     "mla_rope_table_fill": ([_p, _i64, _f64], _i32),
     "mla_absorb_q": ([_p, _p, _p, _p, _p, _i64, _i32, _i32, _p, _p, _p], _i32),
+    "mla_query_up": ([_p, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p], _i32),
     "mla_append_cache": ([_p, _i64, _p, _p, _p, _p, _p, _p, _i64, _i32, _p, _p], _i32),
     "mla_decode_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
     "mla_decode": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
@@ -106,6 +107,22 @@ def absorb_q(q_nope, q_rope, pos, W_UK, rope_tab, q_out=None, dev_status=None, s
         T, H, _ptr(q_out, torch.bfloat16, (T, H, D_ROW), "q_out"),
         _ptr(dev_status, torch.int32, None, "dev_status"), _stream(stream)))
     return q_out
+
+
+def query_up(c_q, W_UQ, W_QR, q_nope=None, q_rope=None, dev_status=None, stream=None):
+    """q^C[t, h] = W^UQ_h c^Q_t -> bf16 [T, H, 128] and q^R[t, h] = W^QR_h c^Q_t -> bf16 [T, H, 64] (not rotated)."""
+    T, d_cq = c_q.shape
+    H = W_UQ.shape[0]
+    if q_nope is None:
+        q_nope = torch.empty((T, H, D_H), dtype=torch.bfloat16, device=c_q.device)
+    if q_rope is None:
+        q_rope = torch.empty((T, H, D_R), dtype=torch.bfloat16, device=c_q.device)
+    _check(lib.mla_query_up(
+        _ptr(c_q, torch.bfloat16, (T, d_cq), "c_q"), _ptr(W_UQ, torch.bfloat16, (H, D_H, d_cq), "W_UQ"),
+        _ptr(W_QR, torch.bfloat16, (H, D_R, d_cq), "W_QR"), T, H, d_cq,
+        _ptr(q_nope, torch.bfloat16, (T, H, D_H), "q_nope"), _ptr(q_rope, torch.bfloat16, (T, H, D_R), "q_rope"),
+        _ptr(dev_status, torch.int32, None, "dev_status"), _stream(stream)))
+    return q_nope, q_rope
 
 
 def new_cache(cap_blocks: int, device="cuda") -> torch.Tensor:

@@ -122,6 +122,19 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* p
                                        static_cast<cudaStream_t>(stream)));
 }
 
+mla_status mla_query_up(const void* c_q, const void* W_UQ, const void* W_QR, int T, int H, int d_cq,
+                        void* q_nope, void* q_rope, int32_t* dev_status, mla_stream stream) {
+    if (T < 0) return MLA_ERR_INVALID_ARG;
+    if (H < 1 || H > kMaxHeads || d_cq < 64 || d_cq > 16384 || d_cq % 64 != 0) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MLA_OK;
+    if (!c_q || !W_UQ || !W_QR || !q_nope || !q_rope) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(c_q) || !aligned16(W_UQ) || !aligned16(W_QR) || !aligned16(q_nope) || !aligned16(q_rope))
+        return MLA_ERR_INVALID_ARG;
+    return cuda_status(launch_query_up(static_cast<const uint16_t*>(c_q), static_cast<const uint16_t*>(W_UQ),
+                                       static_cast<const uint16_t*>(W_QR), T, H, d_cq, static_cast<uint16_t*>(q_nope),
+                                       static_cast<uint16_t*>(q_rope), dev_status, static_cast<cudaStream_t>(stream)));
+}
+
 mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int64_t* seq_block, const int32_t* seq_idx,
                             const int32_t* pos, const void* c_kv, const void* k_rope, const float* rope_table,
                             int64_t rope_len, int T, int32_t* dev_status, mla_stream stream) {

@@ -228,5 +228,5 @@ def query_up(c_q: np.ndarray, W_UQ: np.ndarray, W_QR: np.ndarray):
     q^R happens in the absorb step, at the query's position.
     """
     c_q = _f64(c_q)
-    return (np.einsum("hdk,tk->thd", _f64(W_UQ), c_q),
-            np.einsum("hdk,tk->thd", _f64(W_QR), c_q))
+    return (np.einsum("hdk,tk->thd", _f64(W_UQ), c_q, optimize=True),
+            np.einsum("hdk,tk->thd", _f64(W_QR), c_q, optimize=True))

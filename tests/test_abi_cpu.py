@@ -78,6 +78,12 @@ def test_host_validation_rejects_bad_arguments(mla):
     assert L.mla_append_cache(None, 0, None, None, None, None, None, None, 0, 0, None, None) == 0
     assert L.mla_splitkv_combine(fake, fake, 4, 16, 0, None, fake, None, None) == 2
     assert L.mla_splitkv_combine(None, fake, 4, 16, 2, None, fake, None, None) == 1
+    # query up-projection: empty, d_cq not a multiple of 64, no heads, null input
+    assert L.mla_query_up(None, None, None, 0, 16, 1536, None, None, None, None) == 0
+    assert L.mla_query_up(fake, fake, fake, 4, 16, 100, fake, fake, None, None) == 2
+    assert L.mla_query_up(fake, fake, fake, 4, 0, 1536, fake, fake, None, None) == 2
+    assert L.mla_query_up(fake, fake, fake, -1, 16, 1536, fake, fake, None, None) == 1
+    assert L.mla_query_up(None, fake, fake, 4, 16, 1536, fake, fake, None, None) == 1
 
 
 def test_workspace_sizes(mla):
