@@ -57,6 +57,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-query-up", action="store_true",
+                    help="skip the separate timing of the compressed-query up-projection")
+    ap.add_argument("--query-rank", type=int, default=1536, help="d_c' of the query up-projection timing")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
     return ap.parse_args()
 
@@ -324,6 +327,43 @@ def run_step(mla, cfg, st):
         f(mla, cfg, st)
 
 
+def measure_query_up(torch, mla, cfg, dev, time_graph, n, peaks, d_cq):
+    """Time mla_query_up (c^Q [T, d_c'] -> q^C, q^R) alone, as a CUDA graph after an L2 flush.
+
+    It is the step before absorb_q when queries are compressed, and is not part of the step above.
+    Algorithmic bytes: the weights H*192*d_c'*2, the c^Q rows in and q^C, q^R out.
+    """
+    cq, wuq, wqr = mi.compressed_queries(cfg, d_cq)
+
+    def dbf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    cq_d, wuq_d, wqr_d = dbf(cq), dbf(wuq), dbf(wqr)
+    T, H = cfg.T, cfg.H
+    qn = torch.empty((T, H, mi.D_H), dtype=torch.bfloat16, device=dev)
+    qr = torch.empty((T, H, mi.D_R), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    run = lambda: mla.query_up(cq_d, wuq_d, wqr_d, q_nope=qn, q_rope=qr, dev_status=status)
+    for _ in range(3):
+        run()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        run()
+    torch.cuda.synchronize()
+    ms = time_graph(g, n)
+    torch.cuda.synchronize()
+    del g
+    if int(status.item()) != 0:
+        return {"error": "device status " + mla.device_status_string(int(status.item()))}
+    nbytes = H * (mi.D_H + mi.D_R) * d_cq * 2 + T * d_cq * 2 + T * H * (mi.D_H + mi.D_R) * 2
+    us = 1e3 * statistics.mean(ms)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"kernel": "mla_query_up", "d_cq": d_cq, "T": T, "H": H, "launches": n, "us_per_launch": round(us, 3),
+            "algorithmic_bytes": nbytes, "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "note": "timed alone, L2 flushed before each launch; not part of the step"}
+
+
 def run_ours(args, dist):
     import torch
     dist.init(torch)
@@ -438,6 +478,13 @@ def run_ours(args, dist):
             max(t_bytes, counts["core_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)) / core_s, 4),
     }
     step_roof_s = max(counts["step_bytes"] / (peaks["hbm_gbs"] * 1e9), counts["step_flops"] / (peaks["bf16_tflops"] * 1e12))
+    query_up = None
+    if dist.world == 1 and not args.no_query_up:
+        try:
+            query_up = measure_query_up(torch, mla, cfg, dev, time_graph, min(args.steps, 1000), peaks,
+                                        args.query_rank)
+        except Exception as e:  # reported in the line; the step's numbers above stand on their own
+            query_up = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
@@ -459,6 +506,8 @@ def run_ours(args, dist):
         "gpu_launches": sum(KERNELS_PER_STEP.values()) * args.steps,
         "clocks": clocks,
     }
+    if query_up is not None:
+        line["query_up"] = query_up
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, st["lengths"], counts, args.cpu_seconds)
     dist.close()

@@ -1,0 +1,47 @@
+"""Host-side arithmetic of bench.py, checked on the CPU with stand-ins for the device calls."""
+
+import contextlib
+import os
+import sys
+import types
+
+import numpy as np
+import torch
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+import mla_inputs as mi  # noqa: E402
+
+
+def _fake_torch():
+    class Graph:
+        def replay(self):
+            pass
+
+    t = types.SimpleNamespace(**{k: getattr(torch, k) for k in ("from_numpy", "empty", "zeros", "bfloat16",
+                                                                 "int16", "int32")})
+    t.cuda = types.SimpleNamespace(CUDAGraph=Graph, synchronize=lambda: None,
+                                   graph=lambda g, capture_error_mode=None: contextlib.nullcontext())
+    return t
+
+
+def test_query_up_measurement_bytes_and_shapes():
+    calls = []
+
+    def query_up(cq, wuq, wqr, q_nope=None, q_rope=None, dev_status=None):
+        calls.append((tuple(cq.shape), tuple(wuq.shape), tuple(wqr.shape), tuple(q_nope.shape),
+                      tuple(q_rope.shape)))
+
+    mla = types.SimpleNamespace(query_up=query_up, device_status_string=str)
+    cfg = mi.MLAConfig("small", B=4, H=8, n_q=2, L=64, seed=5)
+    d_cq = 256
+    us = 2.0
+    r = bench.measure_query_up(_fake_torch(), mla, cfg, "cpu", lambda g, n: [us * 1e-3] * n, 7,
+                               {"hbm_gbs": 1000.0}, d_cq)
+    T, H = cfg.T, cfg.H
+    assert calls[0] == ((T, d_cq), (H, 128, d_cq), (H, 64, d_cq), (T, H, 128), (T, H, 64))
+    want = H * 192 * d_cq * 2 + T * d_cq * 2 + T * H * 192 * 2
+    assert r["algorithmic_bytes"] == want
+    assert r["launches"] == 7 and r["us_per_launch"] == us
+    assert np.isclose(r["achieved"], want / (us * 1e-6) / 1e9, rtol=1e-3)
+    assert np.isclose(r["frac"], r["achieved"] / 1000.0, rtol=1e-3)
