@@ -13,6 +13,14 @@
  *   - DeepSeek-V2 MLA explainer (xinfinite.net), section 2.2.2: decoupled
  *     RoPE with per-head q^R and one shared k^R; the RoPE'd key part is cached
  *     so keys need no rotation at inference; attention on [q^C; q^R].[k^C; k^R].
+ *   - The same explainer, section 2.2.1.2: queries are compressed too, to c^Q,
+ *     and up-projected (mla_query_up produces q^C and q^R from c^Q).
+ *
+ * Entry points, in the order a decode step uses them: mla_query_up (when
+ * queries are compressed), mla_absorb_q, mla_append_cache, mla_decode (=
+ * mla_decode_attend + mla_decode_finish; mla_decode_static without a
+ * workspace), with mla_decode_cudacore + mla_splitkv_combine as an
+ * independent CUDA-core path of the same decode.
  *
  * Fixed sizes: d_c = 512, d_h^R = 64, d_h = 128 (cached row D = 576).
  * Runtime sizes: B sequences, H heads (1..128), n_q new query tokens per
