@@ -45,3 +45,25 @@ def test_query_up_measurement_bytes_and_shapes():
     assert r["launches"] == 7 and r["us_per_launch"] == us
     assert np.isclose(r["achieved"], want / (us * 1e-6) / 1e9, rtol=1e-3)
     assert np.isclose(r["frac"], r["achieved"] / 1000.0, rtol=1e-3)
+
+
+def test_reference_arm_line_carries_the_contract_keys():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints one JSON line with the
+    contract's keys, its own cpu_baseline and an e2e object with no host-device traffic."""
+    import json
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0", "--config", "tiny"], cwd=root, capture_output=True, text=True,
+                         timeout=300, check=True).stdout
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"].startswith("tiny")
