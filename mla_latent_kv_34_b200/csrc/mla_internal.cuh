@@ -56,8 +56,6 @@ cudaError_t launch_absorb_tc(const uint16_t* q_nope, const uint16_t* q_rope, con
                              int32_t* dev_status, cudaStream_t stream);
 
 // Query up-projections q^C = W^UQ c^Q, q^R = W^QR c^Q (query_up.cu).
-int query_up_token_block();
-int query_up_mma_n(int T);
 cudaError_t launch_query_up(const uint16_t* c_q, const uint16_t* W_UQ, const uint16_t* W_QR, int T, int H, int d_cq,
                             uint16_t* q_nope, uint16_t* q_rope, int32_t* dev_status, cudaStream_t stream);
 

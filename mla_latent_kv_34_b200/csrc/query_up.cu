@@ -193,15 +193,14 @@ bool matrix_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace qup
+// MMA N (and token rows per TMA box) for T tokens: a multiple of 16, at most one token block.
+int mma_n(int T) { return T >= kTokBlock ? kTokBlock : ((T + 15) & ~15); }
 
-// Tokens per CTA of the query up-projection, and the MMA N it uses for T tokens.
-int query_up_token_block() { return qup::kTokBlock; }
-int query_up_mma_n(int T) { return T >= qup::kTokBlock ? qup::kTokBlock : ((T + 15) & ~15); }
+}  // namespace qup
 
 cudaError_t launch_query_up(const uint16_t* c_q, const uint16_t* W_UQ, const uint16_t* W_QR, int T, int H, int d_cq,
                             uint16_t* q_nope, uint16_t* q_rope, int32_t* dev_status, cudaStream_t stream) {
-    const int NT = query_up_mma_n(T);
+    const int NT = qup::mma_n(T);
     CUtensorMap uq, qr, cq;
     if (!qup::matrix_map(&uq, W_UQ, static_cast<uint64_t>(H) * 128, d_cq, 128) ||
         !qup::matrix_map(&qr, W_QR, static_cast<uint64_t>(H) * 64, d_cq, 64) ||
