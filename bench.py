@@ -9,11 +9,14 @@ tensors of the configuration's shapes (mla_inputs); the cache is filled before
 timing and stays resident in HBM.  L2 is flushed (a 256 MiB write) between
 timed steps.
 
-  python bench.py [--config v2] [--gpus N --steps K --warmup W] [--impl reference]
+  python bench.py [--config ragged] [--gpus N --steps K --warmup W] [--impl reference]
 
-Prints one JSON line (rank 0).  With --gpus N > 1 (torchrun), every rank runs
-its own batch (weak scaling, no data-path collective); timing is the max over
-ranks.  --impl reference times the fp64 CPU oracle on a bounded sample.
+Prints one JSON line (rank 0).  The headline workload is the ragged serving
+batch (the largest single-GPU configuration); at N = 1 the other 128-head
+workloads (V2-shaped and 128K) are measured the same way into `per_config`.
+With --gpus N > 1 (torchrun), every rank runs its own batch (weak scaling, no
+data-path collective); timing is the max over ranks.  --impl reference times
+the fp64 CPU oracle on bounded samples of the same workload.
 """
 
 from __future__ import annotations
@@ -22,8 +25,8 @@ import argparse
 import datetime
 import hashlib
 import json
-import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -43,37 +46,45 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernels each C-ABI call of the step launches
 KERNELS_PER_STEP = {"append": 1, "absorb": 1, "attend": 1, "finish": 1}
 CORE_SOURCES = ["mla_latent_kv_34_b200/csrc/decode_tc.cu", "mla_latent_kv_34_b200/csrc/sm100.cuh"]
+CLOCK_WINDOW_S = 1.0   # the clock sampler needs about a second of load to see several samples
+ORACLE_HEADS = 16      # heads per oracle sample (both the cpu_baseline and the reference arm)
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default 3000 for the CUDA path: about a second, so the clock sampler sees "
-                         "the timed region; 20 oracle samples for --impl reference)")
+                    help="timed steps (default 200 for the CUDA path; 20 oracle samples for --impl reference)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="v2", choices=sorted(mi.CONFIGS))
+    ap.add_argument("--config", default="ragged", choices=sorted(mi.CONFIGS),
+                    help="headline workload (default: ragged, the largest single-GPU configuration)")
+    ap.add_argument("--extra-configs", default="v2,128k",
+                    help="comma-separated configurations also measured (N=1 only) into the line's per_config "
+                         "object; empty to skip")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-query-up", action="store_true",
                     help="skip the separate timing of the compressed-query up-projection")
     ap.add_argument("--query-rank", type=int, default=1536, help="d_c' of the query up-projection timing")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
-    return ap.parse_args()
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle samples")
+    return ap.parse_args(argv)
 
 
 # ------------------------------------------------------------------ workload arithmetic
 
 def step_counts(cfg: mi.MLAConfig, lengths: np.ndarray) -> dict:
-    """Algorithmic bytes / FLOPs of one step (minimum traffic of the documented calls)."""
+    """Algorithmic bytes / FLOPs of one step: the minimum traffic of the step's inputs and outputs.
+
+    The absorbed query q_abs (written by absorb_q, read by the attend kernel) is an intermediate of
+    this implementation and is not counted; nor are the split partials.
+    """
     H, T, n_q = cfg.H, cfg.T, cfg.n_q
     sum_L = int(lengths.sum())
     cache = sum_L * mi.D_ROW * 2  # cached rows read (block padding is not counted)
     weights = 2 * H * mi.D_H * mi.D_C * 2
     q_in = T * H * (mi.D_H + mi.D_R) * 2
-    q_abs = 2 * T * H * mi.D_ROW * 2            # written by absorb, read by attend
     out = T * H * mi.D_H * 2
     new_rows = T * mi.D_ROW * 2 * 2              # raw rows read + packed rows written
     core_flops = 2 * n_q * H * (mi.D_ROW + mi.D_C) * sum_L
@@ -82,7 +93,7 @@ def step_counts(cfg: mi.MLAConfig, lengths: np.ndarray) -> dict:
         "sum_L": sum_L,
         "core_bytes": cache,                      # per cached token: 1152 B
         "core_flops": core_flops,                 # per cached token: 2 n_q H (576 + 512)
-        "step_bytes": cache + weights + q_in + q_abs + out + new_rows,
+        "step_bytes": cache + weights + q_in + out + new_rows,
         "step_flops": core_flops + proj_flops,
     }
 
@@ -118,10 +129,34 @@ def traffic_for(config_name: str, launch_units: int):
     return float(ent["dram_bytes_per_launch"]) * launch_units / float(ent["units"])
 
 
+def roofline_of(counts: dict, core_ms: float, peaks: dict, peak_src: str, traffic) -> dict:
+    """Roofline of the attend kernel: min(HBM, bf16 tensor) bound, burst peaks (the kernel is timed alone)."""
+    core_s = core_ms * 1e-3
+    t_bytes = counts["core_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_flops = counts["core_flops"] / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_bytes >= t_flops else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = counts["core_bytes"] / core_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = counts["core_flops"] / core_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    return {
+        "kernel": "mla_decode_attend", "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
+        "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} (burst)", "traffic": traffic,
+        "algorithmic_bytes": counts["core_bytes"], "algorithmic_flops": counts["core_flops"],
+        "us_per_launch": round(core_ms * 1e3, 3),
+        "tflops_achieved": round(counts["core_flops"] / core_s / 1e12, 2),
+        "hbm_gbs_achieved": round(counts["core_bytes"] / core_s / 1e9, 1),
+        "frac_vs_sustained_tensor": round(
+            max(t_bytes, counts["core_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)) / core_s, 4),
+    }
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    QUERY = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling of SM clocks and throttle reasons; the summary keeps the samples whose
+    timestamps fall inside the window marked by mark_start() / mark_end()."""
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -129,12 +164,12 @@ class ClockSampler:
         self.uuid = uuid
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
-    def start(self, skip: int = 3):
-        self.skip = skip
+    def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
-        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "100"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "50"]
         if self.uuid:
             cmd += ["-i", self.uuid]
         try:
@@ -142,26 +177,27 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+    def mark_start(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
+
+    @staticmethod
+    def parse(lines, t0=None, t1=None):
         rows = []
-        for line in open(self.path):
+        for line in lines:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 10:
                 continue
             try:
-                rows.append({"sm": float(parts[2]), "max": float(parts[3]), "power": float(parts[4]),
-                             "hw": parts[6], "hwt": parts[7], "swt": parts[8], "pcap": parts[9]})
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                row = {"ts": ts, "sm": float(parts[2]), "max": float(parts[3]), "power": float(parts[4]),
+                       "hw": parts[6], "hwt": parts[7], "swt": parts[8], "pcap": parts[9]}
             except ValueError:
                 continue
-        os.unlink(self.path)
-        rows = rows[self.skip:]  # samples taken while the sampler was settling, before the timed region
+            if (t0 is None or ts >= t0) and (t1 is None or ts <= t1):
+                rows.append(row)
         if not rows:
             return None
         reasons = set()
@@ -172,6 +208,19 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["max"] for r in rows),
                 "power_w_max": max(r["power"] for r in rows), "samples": len(rows), "reasons": sorted(reasons)}
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        with open(self.path) as f:
+            lines = f.readlines()
+        os.unlink(self.path)
+        return self.parse(lines, self.t0, self.t1)
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -237,6 +286,11 @@ def aggregate(dist, torch, step_ms: list, step_bytes: float) -> tuple:
     ms_per_step = total_ms / len(step_ms)
     bytes_all = dist.reduce(torch, float(step_bytes), "sum")
     return ms_per_step, bytes_all / (ms_per_step * 1e-3) / 1e12
+
+
+def workload_name(cfg: mi.MLAConfig) -> str:
+    return (f"{cfg.name}: B={cfg.B} H={cfg.H} n_q={cfg.n_q} "
+            f"L={'U[1,%d]' % cfg.L_max if cfg.L is None else cfg.L} d_c=512 d_R=64 d_h=128")
 
 
 # ------------------------------------------------------------------ our arm
@@ -327,6 +381,21 @@ def run_step(mla, cfg, st):
         f(mla, cfg, st)
 
 
+def make_timer(torch, flush):
+    """time_graph(g, n): n replays of graph g, each after an L2 flush, timed by CUDA events on the current
+    stream (the one the graph's launches go to)."""
+    def time_graph(g, n):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            ev[i][0].record()
+            g.replay()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return [e[0].elapsed_time(e[1]) for e in ev]
+    return time_graph
+
+
 def measure_query_up(torch, mla, cfg, dev, time_graph, n, peaks, d_cq):
     """Time mla_query_up (c^Q [T, d_c'] -> q^C, q^R) alone, as a CUDA graph after an L2 flush.
 
@@ -364,31 +433,24 @@ def measure_query_up(torch, mla, cfg, dev, time_graph, n, peaks, d_cq):
             "note": "timed alone, L2 flushed before each launch; not part of the step"}
 
 
-def run_ours(args, dist):
-    import torch
-    dist.init(torch)
-    import mla_latent_kv_34_b200 as mla
-    dev = torch.device("cuda", dist.local_rank)
-    base = mi.CONFIGS[args.config]
-    cfg = rank_config(base, dist.rank)
+def _check_status(mla, st):
+    if int(st["status"].item()) != 0:
+        raise SystemExit(f"device status {mla.device_status_string(int(st['status'].item()))}")
+
+
+def measure_workload(torch, mla, dist, cfg, dev, args, flush, sampler=None, headline=False) -> dict:
+    """Build one workload, then time its step (CUDA graph of the 4 launches), each part alone, and the
+    end-to-end leg through the public API from pinned host buffers.  All timings are CUDA events on the
+    launching stream with an L2 flush before every replay; the step time is the max over ranks."""
     st = build_state(torch, mla, cfg, dev)
     counts = step_counts(cfg, st["lengths"])
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-
+    time_graph = make_timer(torch, flush)
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         run_step(mla, cfg, st)
     torch.cuda.synchronize()
-    if int(st["status"].item()) != 0:
-        raise SystemExit(f"device status {mla.device_status_string(int(st['status'].item()))}")
+    _check_status(mla, st)
 
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-    except Exception:
-        uuid = None
-    sampler = None if args.no_clocks else ClockSampler(uuid)
     # The step is replayed from a CUDA graph (the library's calls neither allocate nor synchronise), so
     # the device runs its launches back to back and host launch overhead stays out of the numbers.
     # Each kernel is also captured alone and timed the same way for the per-kernel split.
@@ -401,38 +463,30 @@ def run_ours(args, dist):
     g_step = capture(lambda: run_step(mla, cfg, st))
     g_parts = {name: capture(lambda f=f: f(mla, cfg, st)) for name, f in STEP_PARTS.items()}
     torch.cuda.synchronize()
-
-    def time_graph(g, n):
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
-        for i in range(n):
-            flush.zero_()
-            ev[i][0].record()
-            g.replay()
-            ev[i][1].record()
-        torch.cuda.synchronize()
-        return [e[0].elapsed_time(e[1]) for e in ev]
-
     time_graph(g_step, 2)
     dist.barrier(torch)
     torch.cuda.synchronize()
     if sampler:
-        sampler.start()
-        time.sleep(0.3)
+        sampler.mark_start()
+    t_start = time.perf_counter()
     step_ms = time_graph(g_step, args.steps)
+    if sampler:
+        # keep the same load on the GPU until the sampler has seen about a second of it (a short timed
+        # region alone would fall between two nvidia-smi samples); these replays are not timed
+        while time.perf_counter() - t_start < CLOCK_WINDOW_S:
+            time_graph(g_step, 20)
+        sampler.mark_end()
+    loaded_s = time.perf_counter() - t_start
     dist.barrier(torch)
-    clocks = sampler.stop() if sampler else None
     part_ms = {name: time_graph(g, args.steps) for name, g in g_parts.items()}
-    core_ms = part_ms["decode_attend"]
-    kernel_us = {name: round(1e3 * statistics.mean(v), 2) for name, v in part_ms.items()}
-    if int(st["status"].item()) != 0:
-        raise SystemExit(f"device status {mla.device_status_string(int(st['status'].item()))}")
+    _check_status(mla, st)
     del g_step, g_parts
-    core_mean_ms = dist.reduce(torch, statistics.mean(core_ms), "max")
+    core_ms = dist.reduce(torch, statistics.mean(part_ms["decode_attend"]), "max")
     ms_per_step, value = aggregate(dist, torch, step_ms, counts["step_bytes"])
     bytes_all = dist.reduce(torch, float(counts["step_bytes"]), "sum")
     flops_all = dist.reduce(torch, float(counts["step_flops"]), "sum")
+    tokens_all = dist.reduce(torch, float(counts["sum_L"]), "sum")
 
-    # end-to-end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
         h, d = st["host"], st["dev"]
@@ -454,68 +508,113 @@ def run_ours(args, dist):
         e2e_ms = dist.reduce(torch, sum(e[0].elapsed_time(e[1]) for e in ee), "max") / args.steps
         e2e = {"value": round(bytes_all / (e2e_ms * 1e-3) / 1e12, 4), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
-    if int(st["status"].item()) != 0:
-        raise SystemExit(f"device status {mla.device_status_string(int(st['status'].item()))}")
+    _check_status(mla, st)
 
     peaks, peak_src = load_peaks()
-    core_s = core_mean_ms * 1e-3
-    t_bytes = counts["core_bytes"] / (peaks["hbm_gbs"] * 1e9)
-    t_flops = counts["core_flops"] / (peaks["bf16_tflops"] * 1e12)
-    bound = "hbm" if t_bytes >= t_flops else "tensor"
-    if bound == "hbm":
-        achieved, peak, unit = counts["core_bytes"] / core_s / 1e9, peaks["hbm_gbs"], "GB/s"
-    else:
-        achieved, peak, unit = counts["core_flops"] / core_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    roofline = {
-        "kernel": "mla_decode_attend", "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-        "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} (burst)",
-        "traffic": traffic_for(args.config, counts["sum_L"]),
-        "algorithmic_bytes": counts["core_bytes"], "algorithmic_flops": counts["core_flops"],
-        "us_per_launch": round(core_mean_ms * 1e3, 3),
-        "tflops_achieved": round(counts["core_flops"] / core_s / 1e12, 2),
-        "hbm_gbs_achieved": round(counts["core_bytes"] / core_s / 1e9, 1),
-        "frac_vs_sustained_tensor": round(
-            max(t_bytes, counts["core_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)) / core_s, 4),
+    roofline = roofline_of(counts, core_ms, peaks, peak_src, traffic_for(cfg.name, counts["sum_L"]))
+    step_roof_s = max(counts["step_bytes"] / (peaks["hbm_gbs"] * 1e9),
+                      counts["step_flops"] / (peaks["bf16_tflops"] * 1e12))
+    res = {
+        "workload": workload_name(cfg), "lengths": st["lengths"], "counts": counts,
+        "ms_per_step": ms_per_step, "value": value, "loaded_s": loaded_s,
+        "us_per_step": round(ms_per_step * 1e3, 2),
+        "kernel_us": {name: round(1e3 * statistics.mean(v), 2) for name, v in part_ms.items()},
+        "tflops": round(flops_all / (ms_per_step * 1e-3) / 1e12, 2),
+        "cache_tokens_per_s": round(tokens_all / (ms_per_step * 1e-3), 1),
+        "step_roofline_frac": round(step_roof_s / (ms_per_step * 1e-3), 4),
+        "roofline": roofline, "e2e": e2e,
     }
-    step_roof_s = max(counts["step_bytes"] / (peaks["hbm_gbs"] * 1e9), counts["step_flops"] / (peaks["bf16_tflops"] * 1e12))
-    query_up = None
-    if dist.world == 1 and not args.no_query_up:
+    if headline and dist.world == 1 and not args.no_query_up:
         try:
-            query_up = measure_query_up(torch, mla, cfg, dev, time_graph, min(args.steps, 1000), peaks,
-                                        args.query_rank)
+            res["query_up"] = measure_query_up(torch, mla, cfg, dev, time_graph, min(args.steps, 1000), peaks,
+                                               args.query_rank)
         except Exception as e:  # reported in the line; the step's numbers above stand on their own
-            query_up = {"error": f"{type(e).__name__}: {e}"[:300]}
+            res["query_up"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    del st
+    torch.cuda.empty_cache()
+    return res
 
+
+def run_ours(args, dist):
+    import torch
+    dist.init(torch)
+    import mla_latent_kv_34_b200 as mla
+    dev = torch.device("cuda", dist.local_rank)
+    cfg = rank_config(mi.CONFIGS[args.config], dist.rank)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    sampler = None if args.no_clocks else ClockSampler(uuid)
+    if sampler:
+        sampler.start()
+    try:
+        head = measure_workload(torch, mla, dist, cfg, dev, args, flush, sampler, headline=True)
+    finally:
+        clocks = sampler.stop() if sampler else None
+    if clocks is not None:
+        clocks["window"] = (f"the timed steps plus untimed replays of the same step graph, "
+                            f"{head['loaded_s']:.2f} s of load in all")
+    per_config = {}
+    extras = [c for c in args.extra_configs.split(",") if c and c != args.config] if dist.world == 1 else []
+    for name in extras:
+        r = measure_workload(torch, mla, dist, rank_config(mi.CONFIGS[name], dist.rank), dev, args, flush)
+        per_config[name] = {k: r[k] for k in ("workload", "us_per_step", "kernel_us", "tflops",
+                                              "cache_tokens_per_s", "step_roofline_frac", "roofline", "e2e")}
+        per_config[name]["value"] = round(r["value"], 4)
+        per_config[name]["unit"] = UNIT
+
+    counts = head["counts"]
     line = {
-        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, mla_inputs)",
-        "config": {"workload": f"{cfg.name}: B={cfg.B} H={cfg.H} n_q={cfg.n_q} "
-                               f"L={'U[1,%d]' % cfg.L_max if cfg.L is None else cfg.L} d_c=512 d_R=64 d_h=128",
-                   "B": cfg.B, "H": cfg.H, "n_q": cfg.n_q, "sum_L": counts["sum_L"],
+        "metric": METRIC, "value": round(head["value"], 4), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(head["ms_per_step"], 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, mla_inputs)",
+        "config": {"workload": head["workload"], "B": cfg.B, "H": cfg.H, "n_q": cfg.n_q, "sum_L": counts["sum_L"],
                    "step": "append + absorb_q + decode_attend + decode_finish",
                    "l2": "flushed between timed steps (256 MiB write)",
-                   "launch": "each timed step is one CUDA graph replay of the 4 library launches", "parallelism": f"dp{args.gpus} (replicas)"},
-        "us_per_step": round(ms_per_step * 1e3, 2),
-        "kernel_us": kernel_us,
-        "tflops": round(flops_all / (ms_per_step * 1e-3) / 1e12, 2),
-        "cache_tokens_per_s": round(dist.reduce(torch, float(counts["sum_L"]), "sum") / (ms_per_step * 1e-3), 1),
-        "step_roofline_frac": round(step_roof_s / (ms_per_step * 1e-3), 4),
-        "roofline": roofline,
-        "e2e": e2e,
+                   "launch": "each timed step is one CUDA graph replay of the 4 library launches",
+                   "parallelism": f"dp{args.gpus} (replicas)"},
+        "us_per_step": head["us_per_step"], "kernel_us": head["kernel_us"], "tflops": head["tflops"],
+        "cache_tokens_per_s": head["cache_tokens_per_s"], "step_roofline_frac": head["step_roofline_frac"],
+        "roofline": head["roofline"], "e2e": head["e2e"],
         "gpu_launches": sum(KERNELS_PER_STEP.values()) * args.steps,
         "clocks": clocks,
     }
-    if query_up is not None:
-        line["query_up"] = query_up
+    if per_config:
+        line["per_config"] = per_config
+    if "query_up" in head:
+        line["query_up"] = head["query_up"]
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, st["lengths"], counts, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(cfg, head["lengths"], args.cpu_seconds)
     dist.close()
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ the oracle as baseline / reference arm
+#
+# Both the cpu_baseline of our line and the reference arm time the SAME thing: the fp64 naive oracle on
+# samples of the workload, each sample = one sequence, a block of ORACLE_HEADS heads, all its query
+# tokens.  Samples cycle through the sequences (and head blocks) in a fixed order.  The oracle's cost is
+# linear in (cached tokens x heads); its rate over the samples gives the full step's time, and `value` is
+# the step's algorithmic bytes over that time (the same unit as our arm's value).
+
+def cpu_info() -> dict:
+    model = platform.processor() or ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count() or 1, "cpu_model": model}
+
 
 def _blas_threads() -> int:
     try:
@@ -526,61 +625,92 @@ def _blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(cfg, lengths, heads, b=0):
-    """Run the fp64 naive oracle on sequence b, the given heads; returns seconds."""
-    from oracle import naive as on
-    s = mi.sequence(cfg, b, lengths)
-    f = mi.bf16_bits_to_f64
-    Wk, Wv = f(mi.weights(cfg, "uk")), f(mi.weights(cfg, "uv"))
-    args = (f(s.c_kv), f(s.k_rope), f(s.q_nope), f(s.q_rope), Wk, Wv, cfg.n_q)
-    t = time.perf_counter()
-    on.attend_naive(*args, scale=cfg.scale, base=cfg.rope_base, heads=heads)
-    return time.perf_counter() - t
+def oracle_sample_plan(cfg: mi.MLAConfig, lengths: np.ndarray, i: int) -> tuple:
+    """Sample i: (sequence, heads).  Sequences in index order, then the next head block."""
+    b = i % cfg.B
+    nh = min(ORACLE_HEADS, cfg.H)
+    h0 = (nh * (i // cfg.B)) % cfg.H
+    heads = [(h0 + k) % cfg.H for k in range(nh)]
+    return b, heads
 
 
-def cpu_baseline(cfg, lengths, counts, target_s: float):
-    b = int(np.argmax(lengths))
-    t1 = oracle_sample(cfg, lengths, [0], b)
-    nh = int(max(1, min(cfg.H, target_s / max(t1, 1e-6))))
-    heads = list(range(nh))
-    t = oracle_sample(cfg, lengths, heads, b)
-    # extrapolate per (cached token x head): the oracle's cost is linear in both
-    per_unit = t / (int(lengths[b]) * nh)
+class OracleTimer:
+    """Times the fp64 naive oracle on samples of one workload (weights widened once)."""
+
+    def __init__(self, cfg: mi.MLAConfig, lengths: np.ndarray):
+        self.cfg, self.lengths = cfg, lengths
+        f = mi.bf16_bits_to_f64
+        self.Wk, self.Wv = f(mi.weights(cfg, "uk")), f(mi.weights(cfg, "uv"))
+
+    def sample(self, i: int) -> tuple:
+        """Returns (seconds, units = cached tokens x heads) of sample i."""
+        from oracle import naive as on
+        cfg = self.cfg
+        b, heads = oracle_sample_plan(cfg, self.lengths, i)
+        s = mi.sequence(cfg, b, self.lengths)
+        f = mi.bf16_bits_to_f64
+        args = (f(s.c_kv), f(s.k_rope), f(s.q_nope), f(s.q_rope), self.Wk, self.Wv, cfg.n_q)
+        t = time.perf_counter()
+        on.attend_naive(*args, scale=cfg.scale, base=cfg.rope_base, heads=heads)
+        return time.perf_counter() - t, int(self.lengths[b]) * len(heads)
+
+
+def oracle_rate_line(cfg, lengths, secs: list, units: list) -> dict:
+    counts = step_counts(cfg, lengths)
+    per_unit = sum(secs) / max(sum(units), 1)
     full_s = per_unit * counts["sum_L"] * cfg.H
-    return {"value": round(counts["step_bytes"] / full_s / 1e12, 8), "unit": UNIT, "cores": _blas_threads(),
-            "kind": "oracle",
-            "sample": f"sequence {b} (L={int(lengths[b])}), {nh}/{cfg.H} heads, {t:.1f} s; "
-                      f"extrapolated to the full step per (cached token x head): {full_s:.1f} s/step"}
+    return {"value": counts["step_bytes"] / full_s / 1e12, "full_step_s": full_s,
+            "sample_s": statistics.mean(secs), "n": len(secs)}
+
+
+def cpu_baseline(cfg, lengths, target_s: float):
+    timer = OracleTimer(cfg, lengths)
+    secs, units = [], []
+    t0 = time.perf_counter()
+    i = 0
+    while i < 3 or (time.perf_counter() - t0 < target_s and i < 10 * cfg.B):
+        s, u = timer.sample(i)
+        secs.append(s)
+        units.append(u)
+        i += 1
+    r = oracle_rate_line(cfg, lengths, secs, units)
+    return {"value": round(r["value"], 8), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle", **cpu_info(),
+            "sample": f"fp64 naive oracle on {r['n']} samples (one sequence x {min(ORACLE_HEADS, cfg.H)} heads x "
+                      f"all queries each, {sum(secs):.1f} s); rate per (cached token x head) scaled to the full "
+                      f"step: {r['full_step_s']:.4g} s/step",
+            "extrapolated_full_step_s": round(r["full_step_s"], 4)}
 
 
 def run_reference(args, dist):
     if dist.rank != 0:
         return
-    base = mi.CONFIGS[args.config]
-    cfg = base
+    cfg = mi.CONFIGS[args.config]
     lengths = mi.kv_lengths(cfg)
-    counts = step_counts(cfg, lengths)
-    b = int(np.argmax(lengths))
-    # one step = the oracle on one head of the longest sequence, extrapolated
-    per = []
-    for i in range(args.warmup + args.steps):
-        t = oracle_sample(cfg, lengths, [i % cfg.H], b)
-        if i >= args.warmup:
-            per.append(t / int(lengths[b]))
-    full_s = statistics.mean(per) * counts["sum_L"] * cfg.H
-    value = counts["step_bytes"] / full_s / 1e12
-    sample = (f"per step: oracle on sequence {b} (L={int(lengths[b])}), 1/{cfg.H} heads; "
-              f"extrapolated per (cached token x head) to {full_s:.4g} s/step")
+    timer = OracleTimer(cfg, lengths)
+    for i in range(args.warmup):
+        timer.sample(i)
+    secs, units = [], []
+    for i in range(args.warmup, args.warmup + args.steps):
+        s, u = timer.sample(i)
+        secs.append(s)
+        units.append(u)
+    r = oracle_rate_line(cfg, lengths, secs, units)
+    value = round(r["value"], 8)
+    sample = (f"each step: the fp64 naive oracle on one sequence x {min(ORACLE_HEADS, cfg.H)} heads x all queries "
+              f"(mean {r['sample_s']:.3f} s); rate per (cached token x head) scaled to the full step: "
+              f"{r['full_step_s']:.4g} s/step")
     line = {
-        "metric": METRIC, "value": round(value, 8), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(full_s * 1e3, 3), "higher_is_better": True,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(r["sample_s"] * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, mla_inputs)",
-        "config": {"workload": f"{cfg.name}: B={cfg.B} H={cfg.H} n_q={cfg.n_q} "
-                               f"L={'U[1,%d]' % cfg.L_max if cfg.L is None else cfg.L} d_c=512 d_R=64 d_h=128"},
+        "config": {"workload": workload_name(cfg), "B": cfg.B, "H": cfg.H, "n_q": cfg.n_q,
+                   "sum_L": int(lengths.sum()),
+                   "step": "one bounded oracle sample of the workload (ms_per_step is its measured time)"},
         "impl": "reference",
-        "cpu_baseline": {"value": round(value, 8), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+        "extrapolated_full_step_s": round(r["full_step_s"], 4),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle", **cpu_info(),
                          "sample": sample},
-        "e2e": {"value": round(value, 8), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
@@ -588,7 +718,7 @@ def run_reference(args, dist):
 def main():
     args = parse_args()
     if args.steps is None:
-        args.steps = 20 if args.impl == "reference" else 3000
+        args.steps = 20 if args.impl == "reference" else 200
     dist = Dist(args.gpus)
     if args.impl == "reference":
         run_reference(args, dist)

@@ -67,3 +67,41 @@ def test_reference_arm_line_carries_the_contract_keys():
     assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"].startswith("tiny")
+
+
+def test_clock_window_keeps_only_samples_inside_it():
+    import datetime as dt
+    lines = []
+    t = dt.datetime(2026, 1, 1, 12, 0, 0)
+    for k in range(10):
+        ts = (t + dt.timedelta(milliseconds=100 * k)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        reason = "Active" if k == 9 else "Not Active"
+        lines.append(f"{ts}, 0, {1000 + k}, 1965, 500.0, 0x0, Not Active, Not Active, Not Active, {reason}\n")
+    r = bench.ClockSampler.parse(lines, t + dt.timedelta(milliseconds=250), t + dt.timedelta(milliseconds=650))
+    assert r["samples"] == 4 and r["sm_mhz"] == 1004.5 and r["reasons"] == []
+    r = bench.ClockSampler.parse(lines)
+    assert r["samples"] == 10 and r["reasons"] == ["sw_power_cap"]
+    assert bench.ClockSampler.parse(lines, t + dt.timedelta(seconds=5)) is None
+
+
+def test_step_bytes_count_inputs_and_outputs_only():
+    cfg = mi.CONFIGS["v2"]
+    c = bench.step_counts(cfg, mi.kv_lengths(cfg))
+    T, H = cfg.T, cfg.H
+    want = (c["sum_L"] * 1152 + 2 * H * 128 * 512 * 2 + T * H * 192 * 2 + T * H * 128 * 2 + T * 576 * 4)
+    assert c["step_bytes"] == want
+    assert c["core_flops"] == 2 * H * 1088 * c["sum_L"]
+
+
+def test_both_oracle_arms_sample_the_same_way():
+    """cpu_baseline and the reference arm share one sample plan and one rate definition."""
+    cfg = mi.CONFIGS["ragged"]
+    L = mi.kv_lengths(cfg)
+    plans = [bench.oracle_sample_plan(cfg, L, i) for i in range(2 * cfg.B + 3)]
+    assert [p[0] for p in plans[:cfg.B]] == list(range(cfg.B))
+    assert all(len(h) == bench.ORACLE_HEADS for _, h in plans)
+    assert plans[cfg.B][1][0] == bench.ORACLE_HEADS
+    r = bench.oracle_rate_line(cfg, L, [2.0, 2.0], [1000, 3000])
+    c = bench.step_counts(cfg, L)
+    assert np.isclose(r["full_step_s"], 4.0 / 4000 * c["sum_L"] * cfg.H)
+    assert np.isclose(r["value"], c["step_bytes"] / r["full_step_s"] / 1e12)
