@@ -44,7 +44,7 @@ METRIC = "MLA absorbed decode: µs/step, TB/s & TFLOP/s as % of B200 roofline"
 UNIT = "TB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # kernels each C-ABI call of the step launches
-KERNELS_PER_STEP = {"append": 1, "absorb": 1, "attend": 1, "finish": 1}
+KERNELS_PER_STEP = {"append": 1, "absorb": 1, "attend": 1, "finish": 2}
 CORE_SOURCES = ["mla_latent_kv_34_b200/csrc/decode_tc.cu", "mla_latent_kv_34_b200/csrc/sm100.cuh"]
 CLOCK_WINDOW_S = 1.0   # the clock sampler needs about a second of load to see several samples
 ORACLE_HEADS = 16      # heads per oracle sample (both the cpu_baseline and the reference arm)
@@ -295,14 +295,24 @@ def workload_name(cfg: mi.MLAConfig) -> str:
 
 # ------------------------------------------------------------------ our arm
 
+def block_table(cfg: mi.MLAConfig, lengths: np.ndarray, n_blocks: int, torch, dev):
+    """The pool's blocks handed to the sequences in a seeded random order (a paged cache as a serving
+    runtime leaves it after sequences have come and gone): int32 [B, max_blocks]."""
+    nblk = (lengths + 127) // 128
+    perm = np.random.default_rng(cfg.seed).permutation(n_blocks).astype(np.int32)
+    tab = np.zeros((cfg.B, int(nblk.max())), dtype=np.int32)
+    k = 0
+    for b in range(cfg.B):
+        tab[b, :nblk[b]] = perm[k:k + nblk[b]]
+        k += int(nblk[b])
+    return torch.from_numpy(tab).to(dev)
+
+
 def build_state(torch, mla, cfg: mi.MLAConfig, dev):
     lengths = mi.kv_lengths(cfg)
     starts = mi.seq_starts(lengths)  # rows of the generator's packed pool
     N = int(lengths.sum())
     nblk = (lengths + mla.BLOCK_TOKENS - 1) // mla.BLOCK_TOKENS
-    seq_block = np.zeros(cfg.B, dtype=np.int64)
-    if cfg.B > 1:
-        seq_block[1:] = np.cumsum(nblk[:-1])
 
     def dbf(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
@@ -310,14 +320,14 @@ def build_state(torch, mla, cfg: mi.MLAConfig, dev):
     cache = torch.zeros((int(nblk.sum()), mla.BLOCK_BYTES), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     rope = mla.rope_table(int(lengths.max()), cfg.rope_base, dev)
-    seq_block_t = torch.from_numpy(seq_block).to(dev)
+    table = block_table(cfg, lengths, int(nblk.sum()), torch, dev)
     seq_of_row = np.repeat(np.arange(cfg.B, dtype=np.int32), lengths)
     pos_of_row = (np.arange(N, dtype=np.int64) - np.repeat(starts, lengths)).astype(np.int32)
     chunk = 1 << 18
     for r0 in range(0, N, chunk):
         n = min(chunk, N - r0)
         c, k = mi.token_rows(cfg, r0, n)
-        mla.append_cache(cache, seq_block_t, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
+        mla.append_cache(cache, table, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
                          torch.from_numpy(pos_of_row[r0:r0 + n]).to(dev), dbf(c), dbf(k), rope, status)
     # the step's new tokens: the last n_q rows of every sequence
     new_rows = np.concatenate([starts[b] + lengths[b] - cfg.n_q + np.arange(cfg.n_q) for b in range(cfg.B)])
@@ -337,7 +347,7 @@ def build_state(torch, mla, cfg: mi.MLAConfig, dev):
     devt = {k: v.to(dev) for k, v in host.items()}
     T, H = cfg.T, cfg.H
     st = {
-        "lengths": lengths, "cache": cache, "status": status, "rope": rope, "seq_block": seq_block_t,
+        "lengths": lengths, "cache": cache, "status": status, "rope": rope, "block_table": table,
         "kv_len": torch.from_numpy(lengths.astype(np.int32)).to(dev),
         "W_UK": dbf(mi.weights(cfg, "uk")), "W_UV": dbf(mi.weights(cfg, "uv")),
         "host": host, "dev": devt,
@@ -352,7 +362,7 @@ def build_state(torch, mla, cfg: mi.MLAConfig, dev):
 
 def step_append(mla, cfg, st):
     d = st["dev"]
-    mla.append_cache(st["cache"], st["seq_block"], d["seq_idx"], d["pos"], d["c_kv"], d["k_rope"], st["rope"],
+    mla.append_cache(st["cache"], st["block_table"], d["seq_idx"], d["pos"], d["c_kv"], d["k_rope"], st["rope"],
                      st["status"])
 
 
@@ -363,12 +373,12 @@ def step_absorb(mla, cfg, st):
 
 
 def step_attend(mla, cfg, st):
-    mla.decode_attend(st["q_abs"], st["cache"], st["seq_block"], st["kv_len"], cfg.n_q, cfg.scale, 0, st["ws"],
+    mla.decode_attend(st["q_abs"], st["cache"], st["block_table"], st["kv_len"], cfg.n_q, cfg.scale, 0, st["ws"],
                       dev_status=st["status"])
 
 
 def step_finish(mla, cfg, st):
-    mla.decode_finish(st["seq_block"], st["kv_len"], st["cache"], st["W_UV"], cfg.n_q, 0, st["ws"], st["out"],
+    mla.decode_finish(st["block_table"], st["kv_len"], st["W_UV"], cfg.n_q, 0, st["ws"], st["out"],
                       dev_status=st["status"])
 
 
@@ -439,7 +449,7 @@ def _check_status(mla, st):
 
 
 def measure_workload(torch, mla, dist, cfg, dev, args, flush, sampler=None, headline=False) -> dict:
-    """Build one workload, then time its step (CUDA graph of the 4 launches), each part alone, and the
+    """Build one workload, then time its step (CUDA graph of the 5 launches), each part alone, and the
     end-to-end leg through the public API from pinned host buffers.  All timings are CUDA events on the
     launching stream with an L2 flush before every replay; the step time is the max over ranks."""
     st = build_state(torch, mla, cfg, dev)
@@ -574,9 +584,10 @@ def run_ours(args, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, mla_inputs)",
         "config": {"workload": head["workload"], "B": cfg.B, "H": cfg.H, "n_q": cfg.n_q, "sum_L": counts["sum_L"],
-                   "step": "append + absorb_q + decode_attend + decode_finish",
+                   "step": "append + absorb_q + decode_attend + decode_finish (merge, W^UV)",
+                   "cache": "paged: pool blocks handed to the sequences in a seeded random order",
                    "l2": "flushed between timed steps (256 MiB write)",
-                   "launch": "each timed step is one CUDA graph replay of the 4 library launches",
+                   "launch": "each timed step is one CUDA graph replay of the 5 library launches",
                    "parallelism": f"dp{args.gpus} (replicas)"},
         "us_per_step": head["us_per_step"], "kernel_us": head["kernel_us"], "tflops": head["tflops"],
         "cache_tokens_per_s": head["cache_tokens_per_s"], "step_roofline_frac": head["step_roofline_frac"],

@@ -26,17 +26,30 @@
  * Runtime sizes: B sequences, H heads (1..128), n_q new query tokens per
  * sequence (1..16), T = B * n_q query rows (row t = b * n_q + j).
  *
- * Latent cache layout (blocked).  The cache is an array of blocks of
- * MLA_BLOCK_TOKENS = 128 tokens, MLA_BLOCK_BYTES = 147456 bytes each.  Token
- * `pos` of sequence b lives in block seq_block[b] + pos / 128, at row
- * r = pos % 128; its 576 bf16 values [c^KV (0..511) | rotated k^R (512..575)]
- * are stored as nine 64-column chunks, column c at byte offset
+ * Latent cache layout (paged, blocked).  The cache is a pool of blocks of
+ * MLA_BLOCK_TOKENS = 128 tokens, MLA_BLOCK_BYTES = 147456 bytes each, and a
+ * block table maps each sequence's token positions to pool blocks: token
+ * `pos` of sequence b lives in block block_table[b * max_blocks + pos / 128],
+ * at row r = pos % 128.  A sequence's blocks need not be consecutive or in
+ * any order, so a serving runtime can hand out blocks of one pool as
+ * sequences grow and free them in any order, with no copying and no
+ * fragmentation beyond one partly filled block per sequence (the paged
+ * KV-cache of vLLM/PagedAttention, named as the complementary technique in the
+ * MLA explainer (xinfinite.net), section 2.1.1).  The token's 576 bf16 values
+ * [c^KV (0..511) | rotated k^R (512..575)] are stored as nine 64-column
+ * chunks, column c at byte offset
  *     (c / 64) * 16384 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2
  * within the block: each chunk is a [128 rows x 128 bytes] tile whose 16-byte
  * units are permuted by the row index (the 128-byte swizzle), so that
  * contiguous copies place a block in shared memory exactly as the tensor-core
- * operands are read (128 tokens per block make the score MMA 128 wide).  Each
- * sequence occupies ceil(L_b / 128) consecutive blocks.
+ * operands are read (128 tokens per block make the score MMA 128 wide).
+ *
+ * Block table: int32 [B, max_blocks], row-major, device memory.  Row b lists
+ * the pool blocks of sequence b in position order; only its first
+ * ceil(kv_len[b] / 128) entries are read.  A sequence longer than
+ * max_blocks * 128 tokens is not processed and sets MLA_DEVERR_ROW_RANGE; an
+ * entry read outside [0, cap_blocks) sets MLA_DEVERR_ROW_RANGE and that
+ * sequence's results are unspecified (no access outside the pool is made).
  *
  * Conventions for every entry point:
  *   - All tensor arguments are DEVICE pointers to caller-owned memory, dense
@@ -88,7 +101,7 @@ typedef enum {
 
 const char* mla_status_string(int status);
 const char* mla_device_status_string(int32_t dev_status_word);
-int mla_abi_version(void);
+int mla_abi_version(void); /* 2: paged cache (block tables) */
 
 /*
  * mla_rope_table_fill -- HOST function.  table_host: fp32 [rope_len, 64],
@@ -142,34 +155,43 @@ mla_status mla_query_up(const void* c_q, const void* W_UQ, const void* W_QR, int
                         void* q_nope, void* q_rope, int32_t* dev_status, mla_stream stream);
 
 /*
- * mla_append_cache -- write T new tokens into the blocked latent cache.
+ * mla_append_cache -- write T new tokens into the paged latent cache.
  * ("两张账" page: only c^KV and k^R are cached; explainer 2.2.2: k^R is
  *  cached already rotated.)
- *   cache      cap_blocks blocks of MLA_BLOCK_BYTES (layout above); token i
- *              goes to block seq_block[seq_idx[i]] + pos[i] / 128, row pos[i] % 128
- *   seq_block  int64 [*]  first cache block of each sequence
- *   seq_idx    int32 [T]  sequence of token i
- *   pos        int32 [T]  position of token i within its sequence
- *   c_kv       bf16 [T, 512]   copied to columns 0..511 bit for bit
- *   k_rope     bf16 [T, 64]    rotated at pos[i] into columns 512..575
+ *   cache        pool of cap_blocks blocks of MLA_BLOCK_BYTES (layout above)
+ *   block_table  int32 [num_seqs, max_blocks]  token i goes to pool block
+ *                block_table[seq_idx[i] * max_blocks + pos[i] / 128], row pos[i] % 128
+ *   seq_idx      int32 [T]  sequence of token i
+ *   pos          int32 [T]  position of token i within its sequence
+ *   c_kv         bf16 [T, 512]   copied to columns 0..511 bit for bit
+ *   k_rope       bf16 [T, 64]    rotated at pos[i] into columns 512..575
  * The rotation is y0 = fl(fl(x0 c) - fl(x1 s)), y1 = fl(fl(x0 s) + fl(x1 c))
  * in fp32 (no fused multiply-add) with (c, s) from rope_table, then
  * round-to-nearest-even to bf16: the result is reproducible bit for bit.
- * Out-of-range rows or positions set a MLA_DEVERR_* bit and are skipped.
+ * A token whose sequence is outside [0, num_seqs), whose position is negative
+ * or past its table row (pos / 128 >= max_blocks), or whose table entry lies
+ * outside [0, cap_blocks), sets
+ * MLA_DEVERR_ROW_RANGE and is skipped; a position outside the RoPE table sets
+ * MLA_DEVERR_POS_RANGE and is skipped.  Errors: MLA_ERR_INVALID_ARG for null
+ * or misaligned pointers, negative sizes, num_seqs or max_blocks < 1 (before
+ * any launch).
  */
-mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int64_t* seq_block,
-                            const int32_t* seq_idx, const int32_t* pos, const void* c_kv,
-                            const void* k_rope, const float* rope_table, int64_t rope_len,
-                            int T, int32_t* dev_status, mla_stream stream);
+mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int32_t* block_table,
+                            int num_seqs, int max_blocks, const int32_t* seq_idx, const int32_t* pos,
+                            const void* c_kv, const void* k_rope, const float* rope_table,
+                            int64_t rope_len, int T, int32_t* dev_status, mla_stream stream);
 
 /*
  * mla_decode_workspace_bytes -- device workspace mla_decode needs for these
- * sizes (num_splits as passed to mla_decode; 0 = automatic).
+ * sizes (num_splits as passed to mla_decode; 0 = automatic).  It holds the
+ * attend phase's pieces (a slot of 128 rows x (512 fp32 + max, sum) per
+ * sequence plus one per CTA pair, at most 74 pairs, per group of 128 query
+ * rows) and the merged latent output in bf16 ([H, ~B*n_q, 512]).
  */
 size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
 
 /*
- * mla_decode -- one absorbed MLA decode step over the latent cache.
+ * mla_decode -- one absorbed MLA decode step over the paged latent cache.
  * For every sequence b, query j and head h, with p = kv_len[b] - n_q + j:
  *   s_t   = (q[t,h,:512] . c_t + q[t,h,512:] . k^R_t) * scale,  t = 0..p
  *   P     = softmax(s)                   (fp32, online / split-KV)
@@ -179,10 +201,11 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
  *  latent space, W^UV afterwards; explainer 2.2.2 for the concatenated
  *  content/position inner product.)
  *   q          bf16 [B*n_q, H, 576]   from mla_absorb_q
- *   cache      cap_blocks blocks (layout above); sequence b occupies blocks
- *              seq_block[b] .. seq_block[b] + ceil(kv_len[b] / 128) - 1 (kv_len
- *              counts the n_q tokens of this step, already appended)
- *   seq_block  int64 [B];  kv_len int32 [B]
+ *   cache      pool of cap_blocks blocks (layout above)
+ *   block_table int32 [B, max_blocks]: tile i (tokens 128 i .. 128 i + 127) of
+ *              sequence b is pool block block_table[b * max_blocks + i]
+ *   kv_len     int32 [B]: cached tokens of each sequence, counting the n_q
+ *              tokens of this step (already appended)
  *   W_UV       bf16 [H, 128, 512]
  *   scale      softmax scale, 1/sqrt(d_h + d_h^R) = 1/sqrt(192) for V2 shapes
  *   num_splits 0: use every SM.  n > 0: at most n CTA pairs per group of 128
@@ -193,31 +216,41 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
  *   workspace  device scratch of at least mla_decode_workspace_bytes() bytes
  *   out        bf16 [B*n_q, H, 128]
  *   lse_out    fp32 [B*n_q, H] or NULL: log sum_t exp(s_t)
- * A sequence with kv_len[b] < n_q sets MLA_DEVERR_KV_LEN and its rows are
- * left unwritten; blocks beyond cap_blocks set MLA_DEVERR_ROW_RANGE.
+ * A sequence with kv_len[b] < n_q sets MLA_DEVERR_KV_LEN, one longer than
+ * max_blocks * 128 sets MLA_DEVERR_ROW_RANGE; neither is processed and their
+ * rows get out = 0 and lse = -inf.  A table entry outside [0, cap_blocks) sets
+ * MLA_DEVERR_ROW_RANGE (that sequence's rows are then unspecified).
+ * The call launches the attend kernel, then the merge and up-projection
+ * kernels (mla_decode_finish), each with programmatic stream serialization:
+ * a kernel's set-up may overlap the end of the previous kernel on `stream`,
+ * and it waits for that kernel to complete before reading any input.
+ * Errors: MLA_ERR_INVALID_ARG (null or misaligned pointer, bad scale, cap_blocks
+ * or max_blocks < 1), MLA_ERR_UNSUPPORTED_SHAPE, MLA_ERR_WORKSPACE (ws_bytes
+ * below mla_decode_workspace_bytes()), all before any launch; MLA_ERR_CUDA.
  */
 mla_status mla_decode(const void* q, const void* cache, int64_t cap_blocks,
-                      const int64_t* seq_block, const int32_t* kv_len, const void* W_UV,
-                      int B, int n_q, int H, float scale, int num_splits,
+                      const int32_t* block_table, int max_blocks, const int32_t* kv_len,
+                      const void* W_UV, int B, int n_q, int H, float scale, int num_splits,
                       void* workspace, size_t ws_bytes, void* out, float* lse_out,
                       int32_t* dev_status, mla_stream stream);
 
 /*
  * mla_decode_attend / mla_decode_finish -- the two phases of mla_decode,
  * exposed so that callers can place work (or timing events) between them.
- * attend: scores, online softmax and latent aggregation into per-split
- * partials held in `workspace`; finish: log-sum-exp merge of the partials
- * and the W^UV up-projection into `out` (and `lse_out`).  Arguments mean the
- * same as for mla_decode; both calls must see the same sizes, num_splits and
+ * attend: scores, online softmax and latent aggregation into per-piece
+ * partials held in `workspace` (one kernel); finish: log-sum-exp merge of the
+ * pieces of each sequence (one kernel) and the W^UV up-projection into `out`
+ * and `lse_out` (one kernel).  Arguments mean the same as for mla_decode;
+ * both calls must see the same B, n_q, H, kv_len, max_blocks, num_splits and
  * workspace, and finish must be ordered after attend on the stream.
  */
 mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_blocks,
-                             const int64_t* seq_block, const int32_t* kv_len,
+                             const int32_t* block_table, int max_blocks, const int32_t* kv_len,
                              int B, int n_q, int H, float scale, int num_splits,
                              void* workspace, size_t ws_bytes, int32_t* dev_status,
                              mla_stream stream);
-mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, int64_t cap_blocks,
-                             const void* W_UV, int B, int n_q, int H, int num_splits,
+mla_status mla_decode_finish(const int32_t* kv_len, int max_blocks, const void* W_UV,
+                             int B, int n_q, int H, int num_splits,
                              void* workspace, size_t ws_bytes, void* out, float* lse_out,
                              int32_t* dev_status, mla_stream stream);
 
@@ -232,10 +265,12 @@ mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, in
  *   Arguments, layouts and results are those of mla_decode.
  *   Limit: shapes with mla_decode_workspace_bytes(B, n_q, H, num_splits) >
  *   MLA_DECODE_STATIC_SCRATCH_BYTES return MLA_ERR_WORKSPACE and launch
- *   nothing (with 74 CTA pairs and 128 query rows per group this allows
- *   groups * (B + 74) <= 127, e.g. B <= 53 at H = 128, n_q = 1).
+ *   nothing (for example B <= 32 at H = 128, n_q = 1).
  *   Set-up: the first call on a device looks the buffer up (and may load the
- *   library's device code there); make it before any stream capture.
+ *   library's device code there); make it before any stream capture.  The
+ *   address found is kept for the life of the process: after a reset of the
+ *   device (cudaDeviceReset, or any teardown of its primary context) this
+ *   entry point must not be called again on that device.
  *   Zeroing: none needed; every partial read is written in the same call.
  *   Races: one buffer per device, so calls that can overlap on a device
  *   (other streams, unordered host threads) corrupt each other's partials;
@@ -243,7 +278,8 @@ mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, in
  */
 #define MLA_DECODE_STATIC_SCRATCH_BYTES (32u << 20)
 mla_status mla_decode_static(const void* q, const void* cache, int64_t cap_blocks,
-                             const int64_t* seq_block, const int32_t* kv_len, const void* W_UV,
+                             const int32_t* block_table, int max_blocks, const int32_t* kv_len,
+                             const void* W_UV,
                              int B, int n_q, int H, float scale, int num_splits,
                              void* out, float* lse_out, int32_t* dev_status, mla_stream stream);
 
@@ -257,7 +293,8 @@ mla_status mla_decode_static(const void* q, const void* cache, int64_t cap_block
  */
 size_t mla_decode_cudacore_workspace_bytes(int B, int n_q, int H, int num_splits);
 mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_blocks,
-                               const int64_t* seq_block, const int32_t* kv_len, const void* W_UV,
+                               const int32_t* block_table, int max_blocks, const int32_t* kv_len,
+                               const void* W_UV,
                                int B, int n_q, int H, float scale, int num_splits,
                                void* workspace, size_t ws_bytes, void* out, float* lse_out,
                                int32_t* dev_status, mla_stream stream);

@@ -35,15 +35,15 @@ _SIGS = {
     "mla_rope_table_fill": ([_p, _i64, _f64], _i32),
     "mla_absorb_q": ([_p, _p, _p, _p, _p, _i64, _i32, _i32, _p, _p, _p], _i32),
     "mla_query_up": ([_p, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p], _i32),
-    "mla_append_cache": ([_p, _i64, _p, _p, _p, _p, _p, _p, _i64, _i32, _p, _p], _i32),
+    "mla_append_cache": ([_p, _i64, _p, _i32, _i32, _p, _p, _p, _p, _p, _i64, _i32, _p, _p], _i32),
     "mla_decode_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
-    "mla_decode": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
-    "mla_decode_attend": ([_p, _p, _i64, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p], _i32),
-    "mla_decode_finish": ([_p, _p, _i64, _p, _i32, _i32, _i32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
-    "mla_decode_static": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _p, _p, _p], _i32),
+    "mla_decode": ([_p, _p, _i64, _p, _i32, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
+    "mla_decode_attend": ([_p, _p, _i64, _p, _i32, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p], _i32),
+    "mla_decode_finish": ([_p, _i32, _p, _i32, _i32, _i32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
+    "mla_decode_static": ([_p, _p, _i64, _p, _i32, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _p, _p, _p], _i32),
     "mla_decode_cudacore_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
-    "mla_decode_cudacore": ([_p, _p, _i64, _p, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p],
-                            _i32),
+    "mla_decode_cudacore": ([_p, _p, _i64, _p, _i32, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p,
+                             _p], _i32),
     "mla_splitkv_combine": ([_p, _p, _i32, _i32, _i32, _p, _p, _p, _p], _i32),
 }
 for _name, (_args, _ret) in _SIGS.items():
@@ -126,8 +126,24 @@ def query_up(c_q, W_UQ, W_QR, q_nope=None, q_rope=None, dev_status=None, stream=
 
 
 def new_cache(cap_blocks: int, device="cuda") -> torch.Tensor:
-    """An empty blocked latent cache: uint8 [cap_blocks, BLOCK_BYTES] (layout in include/mla.h)."""
+    """An empty pool of cache blocks: uint8 [cap_blocks, BLOCK_BYTES] (layout in include/mla.h)."""
     return torch.empty((cap_blocks, BLOCK_BYTES), dtype=torch.uint8, device=device)
+
+
+def contiguous_block_table(lengths, max_blocks: int | None = None, first_block: int = 0, gap_blocks: int = 0,
+                           device="cuda") -> torch.Tensor:
+    """int32 [B, max_blocks] table giving each sequence consecutive pool blocks, sequences back to back
+    (``gap_blocks`` apart) from ``first_block``; unused entries are -1."""
+    import numpy as np
+    lengths = np.asarray(lengths, dtype=np.int64)
+    nblk = (lengths + BLOCK_TOKENS - 1) // BLOCK_TOKENS
+    mb = int(max(1, nblk.max() if len(nblk) else 1)) if max_blocks is None else max_blocks
+    tab = np.full((len(lengths), mb), -1, dtype=np.int32)
+    start = first_block
+    for b, n in enumerate(nblk):
+        tab[b, :n] = start + np.arange(n)
+        start += int(n) + gap_blocks
+    return torch.from_numpy(tab).to(device)
 
 
 def _cache_ptr(cache):
@@ -136,11 +152,19 @@ def _cache_ptr(cache):
     return _ptr(cache, torch.uint8, None, "cache")
 
 
-def append_cache(cache, seq_block, seq_idx, pos, c_kv, k_rope, rope_tab, dev_status=None, stream=None):
-    """Write c_kv [T,512] and R_pos k_rope [T,64] at token pos of sequence seq_idx (block seq_block[seq_idx] + pos/128)."""
+def _table(block_table, B=None):
+    if block_table.dim() != 2 or (B is not None and block_table.shape[0] != B):
+        raise MLAError("block_table must be int32 [B, max_blocks]")
+    return _ptr(block_table, torch.int32, None, "block_table"), block_table.shape[1]
+
+
+def append_cache(cache, block_table, seq_idx, pos, c_kv, k_rope, rope_tab, dev_status=None, stream=None):
+    """Write c_kv [T,512] and R_pos k_rope [T,64] at token pos of sequence seq_idx
+    (pool block block_table[seq_idx, pos // 128], row pos % 128)."""
     T = c_kv.shape[0]
+    tp, mb = _table(block_table)
     _check(lib.mla_append_cache(
-        _cache_ptr(cache), cache.shape[0], _ptr(seq_block, torch.int64, None, "seq_block"),
+        _cache_ptr(cache), cache.shape[0], tp, block_table.shape[0], mb,
         _ptr(seq_idx, torch.int32, (T,), "seq_idx"), _ptr(pos, torch.int32, (T,), "pos"),
         _ptr(c_kv, torch.bfloat16, (T, D_C), "c_kv"), _ptr(k_rope, torch.bfloat16, (T, D_R), "k_rope"),
         _ptr(rope_tab, torch.float32, None, "rope_table"), rope_tab.shape[0], T,
@@ -151,7 +175,7 @@ def decode_workspace_bytes(B: int, n_q: int, H: int, num_splits: int = 0) -> int
     return int(lib.mla_decode_workspace_bytes(B, n_q, H, num_splits))
 
 
-def decode(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
+def decode(q, cache, block_table, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
            workspace=None, out=None, lse_out=None, dev_status=None, stream=None):
     """One absorbed decode step: out bf16 [B*n_q, H, 128] (and lse fp32 [B*n_q, H] if given)."""
     B = kv_len.shape[0]
@@ -164,8 +188,8 @@ def decode(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits
     if out is None:
         out = torch.empty((T, H, D_H), dtype=torch.bfloat16, device=q.device)
     _check(lib.mla_decode(
-        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0],
-        _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0], *_table(block_table, B),
+        _ptr(kv_len, torch.int32, (B,), "kv_len"),
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, float(scale), num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(out, torch.bfloat16, (T, H, D_H), "out"), _ptr(lse_out, torch.float32, (T, H), "lse_out"),
@@ -176,7 +200,7 @@ def decode(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits
 DECODE_STATIC_SCRATCH_BYTES = 32 << 20  # MLA_DECODE_STATIC_SCRATCH_BYTES
 
 
-def decode_static(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
+def decode_static(q, cache, block_table, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
                   out=None, lse_out=None, dev_status=None, stream=None):
     """``decode`` with the library's own scratch (no workspace; ``out`` must be given to avoid any allocation).
 
@@ -190,34 +214,34 @@ def decode_static(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num
     if out is None:
         out = torch.empty((T, H, D_H), dtype=torch.bfloat16, device=q.device)
     _check(lib.mla_decode_static(
-        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0],
-        _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0], *_table(block_table, B),
+        _ptr(kv_len, torch.int32, (B,), "kv_len"),
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, float(scale), num_splits,
         _ptr(out, torch.bfloat16, (T, H, D_H), "out"), _ptr(lse_out, torch.float32, (T, H), "lse_out"),
         _ptr(dev_status, torch.int32, None, "dev_status"), _stream(stream)))
     return out
 
 
-def decode_attend(q, cache, seq_block, kv_len, n_q: int, scale: float, num_splits: int, workspace,
+def decode_attend(q, cache, block_table, kv_len, n_q: int, scale: float, num_splits: int, workspace,
                   dev_status=None, stream=None):
-    """Phase 1 of decode: per-split partials into ``workspace``."""
+    """Phase 1 of decode: per-piece partials into ``workspace``."""
     B = kv_len.shape[0]
     T, H = q.shape[0], q.shape[1]
     _check(lib.mla_decode_attend(
         _ptr(q, torch.bfloat16, (B * n_q, H, D_ROW), "q"), _cache_ptr(cache),
-        cache.shape[0], _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        cache.shape[0], *_table(block_table, B), _ptr(kv_len, torch.int32, (B,), "kv_len"),
         B, n_q, H, float(scale), num_splits, _ptr(workspace, None, None, "workspace"),
         workspace.numel() * workspace.element_size(), _ptr(dev_status, torch.int32, None, "dev_status"),
         _stream(stream)))
 
 
-def decode_finish(seq_block, kv_len, cache, W_UV, n_q: int, num_splits: int, workspace, out, lse_out=None,
+def decode_finish(block_table, kv_len, W_UV, n_q: int, num_splits: int, workspace, out, lse_out=None,
                   dev_status=None, stream=None):
-    """Phase 2 of decode: merge the partials, apply W^UV into ``out`` bf16 [B*n_q, H, 128]."""
+    """Phase 2 of decode: merge the pieces, apply W^UV into ``out`` bf16 [B*n_q, H, 128]."""
     B = kv_len.shape[0]
     H = W_UV.shape[0]
     _check(lib.mla_decode_finish(
-        _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"), cache.shape[0],
+        _ptr(kv_len, torch.int32, (B,), "kv_len"), block_table.shape[1],
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(out, torch.bfloat16, (B * n_q, H, D_H), "out"), _ptr(lse_out, torch.float32, (B * n_q, H), "lse_out"),
@@ -225,7 +249,7 @@ def decode_finish(seq_block, kv_len, cache, W_UV, n_q: int, num_splits: int, wor
     return out
 
 
-def decode_cudacore(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
+def decode_cudacore(q, cache, block_table, kv_len, W_UV, n_q: int, scale: float, num_splits: int = 0,
                     workspace=None, out=None, lse_out=None, dev_status=None, stream=None):
     """The decode step on CUDA cores (second implementation, same results within fp32 rounding)."""
     B = kv_len.shape[0]
@@ -238,8 +262,8 @@ def decode_cudacore(q, cache, seq_block, kv_len, W_UV, n_q: int, scale: float, n
     if out is None:
         out = torch.empty((T, H, D_H), dtype=torch.bfloat16, device=q.device)
     _check(lib.mla_decode_cudacore(
-        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0],
-        _ptr(seq_block, torch.int64, (B,), "seq_block"), _ptr(kv_len, torch.int32, (B,), "kv_len"),
+        _ptr(q, torch.bfloat16, (T, H, D_ROW), "q"), _cache_ptr(cache), cache.shape[0], *_table(block_table, B),
+        _ptr(kv_len, torch.int32, (B,), "kv_len"),
         _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), B, n_q, H, float(scale), num_splits,
         _ptr(workspace, None, None, "workspace"), workspace.numel() * workspace.element_size(),
         _ptr(out, torch.bfloat16, (T, H, D_H), "out"), _ptr(lse_out, torch.float32, (T, H), "lse_out"),

@@ -7,23 +7,29 @@
 // (__fmul_rn / __fadd_rn / __fsub_rn are never contracted into an FMA), then
 // round-to-nearest-even to bf16, so the stored bits are reproducible.
 //
-// Block layout (see mla.h): row r of a 128-token block keeps column c at byte
+// Paged layout (see mla.h): token pos of sequence s is row pos % 128 of pool block
+// block_table[s][pos / 128]; row r of a block keeps column c at byte
 // (c / 64) * 16384 + r * 128 + (((c % 64) / 8) ^ (r % 8)) * 16 + (c % 8) * 2.
 #include "mla_internal.cuh"
 
 namespace mla {
 
 __global__ void __launch_bounds__(256) append_cache_kernel(
-    uint8_t* __restrict__ cache, int64_t cap_blocks, const int64_t* __restrict__ seq_block,
-    const int32_t* __restrict__ seq_idx, const int32_t* __restrict__ pos,
+    uint8_t* __restrict__ cache, int64_t cap_blocks, const int32_t* __restrict__ block_table, int num_seqs,
+    int max_blocks, const int32_t* __restrict__ seq_idx, const int32_t* __restrict__ pos,
     const uint16_t* __restrict__ c_kv, const uint16_t* __restrict__ k_rope,
     const float* __restrict__ rope_table, int64_t rope_len, int T, int32_t* dev_status) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= T) return;
     const int32_t p = pos[warp];
-    const int64_t blk = seq_block[seq_idx[warp]] + (p >= 0 ? p / kBlockTokens : 0);
-    if (p < 0 || blk < 0 || blk >= cap_blocks) {
+    const int32_t sq = seq_idx[warp];
+    // the sequence's block-table entry for this position; sequences outside the table, positions past
+    // the row, negative indices and entries outside the pool are reported and skipped
+    int64_t blk = -1;
+    if (p >= 0 && sq >= 0 && sq < num_seqs && p / kBlockTokens < max_blocks)
+        blk = block_table[static_cast<int64_t>(sq) * max_blocks + p / kBlockTokens];
+    if (blk < 0 || blk >= cap_blocks) {
         if (lane == 0) report(dev_status, MLA_DEVERR_ROW_RANGE);
         return;
     }
@@ -52,14 +58,16 @@ __global__ void __launch_bounds__(256) append_cache_kernel(
     *reinterpret_cast<uint32_t*>(dst + 8 * kBlockChunk + ((u ^ (r & 7)) << 4) + (lane & 3) * 4) = pack_bf16x2(y0, y1);
 }
 
-cudaError_t launch_append_cache(uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block, const int32_t* seq_idx,
-                                const int32_t* pos, const uint16_t* c_kv, const uint16_t* k_rope,
-                                const float* rope_table, int64_t rope_len, int T, int32_t* dev_status,
-                                cudaStream_t stream) {
+cudaError_t launch_append_cache(uint8_t* cache, int64_t cap_blocks, const int32_t* block_table, int num_seqs,
+                                int max_blocks,
+                                const int32_t* seq_idx, const int32_t* pos, const uint16_t* c_kv,
+                                const uint16_t* k_rope, const float* rope_table, int64_t rope_len, int T,
+                                int32_t* dev_status, cudaStream_t stream) {
     const int threads = 256;
     const int64_t blocks = (static_cast<int64_t>(T) * 32 + threads - 1) / threads;
     append_cache_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        cache, cap_blocks, seq_block, seq_idx, pos, c_kv, k_rope, rope_table, rope_len, T, dev_status);
+        cache, cap_blocks, block_table, num_seqs, max_blocks, seq_idx, pos, c_kv, k_rope, rope_table, rope_len, T,
+        dev_status);
     return cudaGetLastError();
 }
 

@@ -40,7 +40,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __global__ void __launch_bounds__(256) decode_simt_kernel(
     const uint16_t* __restrict__ q, const uint8_t* __restrict__ cache, int64_t cap_blocks,
-    const int64_t* __restrict__ seq_block, const int32_t* __restrict__ kv_len, int n_q, int H,
+    const int32_t* __restrict__ block_table, int max_blocks, const int32_t* __restrict__ kv_len, int n_q, int H,
     float scale_log2, int S, float* __restrict__ o_part, float* __restrict__ lse_part, int32_t* dev_status) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SimtSmem& sm = *reinterpret_cast<SimtSmem*>(smem_raw);
@@ -51,12 +51,12 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
     const int nrows = min(kSimtRows, R - r0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int L = kv_len[b];
-    const int64_t blk0 = seq_block[b];
+    const int32_t* tab = block_table + static_cast<int64_t>(b) * max_blocks;
     if (L < n_q) {
         if (tid == 0 && s == 0 && blockIdx.y == 0) report(dev_status, MLA_DEVERR_KV_LEN);
         return;
     }
-    if (blk0 < 0 || blk0 + (L + kBlockTokens - 1) / kBlockTokens > cap_blocks) {
+    if ((L + kBlockTokens - 1) / kBlockTokens > max_blocks) {
         if (tid == 0 && s == 0 && blockIdx.y == 0) report(dev_status, MLA_DEVERR_ROW_RANGE);
         return;
     }
@@ -88,10 +88,16 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
         for (int idx = tid; idx < kSimtTok * (kRow / 2); idx += blockDim.x) {
             const int tk = idx / (kRow / 2), w = idx % (kRow / 2);
             const int t = ts + tk;
-            sm.kv[tk][w] = (t < t_hi) ? *reinterpret_cast<const uint32_t*>(
-                                            cache + (blk0 + t / kBlockTokens) * kBlockBytes +
-                                            block_offset(t % kBlockTokens, 2 * w))
-                                      : 0u;
+            uint32_t v = 0u;
+            if (t < t_hi) {
+                int64_t e = tab[t / kBlockTokens];
+                if (e < 0 || e >= cap_blocks) {  // outside the pool: reported, block 0 read instead
+                    if (w == 0) report(dev_status, MLA_DEVERR_ROW_RANGE);
+                    e = 0;
+                }
+                v = *reinterpret_cast<const uint32_t*>(cache + e * kBlockBytes + block_offset(t % kBlockTokens, 2 * w));
+            }
+            sm.kv[tk][w] = v;
         }
         __syncthreads();
         // scores: lane = token, two rows per warp
@@ -156,8 +162,8 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(
     }
 }
 
-cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
-                               const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,
+cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
+                               int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,
                                float* o_part, float* lse_part, int32_t* dev_status, cudaStream_t stream) {
     const int R = n_q * H;
     dim3 grid(splits, (R + kSimtRows - 1) / kSimtRows, B);
@@ -166,7 +172,8 @@ cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t 
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const float scale_log2 = scale * 1.44269504088896340736f;
-    decode_simt_kernel<<<grid, 256, smem, stream>>>(q, cache, cap_blocks, seq_block, kv_len, n_q, H, scale_log2, splits,
+    decode_simt_kernel<<<grid, 256, smem, stream>>>(q, cache, cap_blocks, block_table, max_blocks, kv_len, n_q, H,
+                                                    scale_log2, splits,
                                                     o_part, lse_part, dev_status);
     return cudaGetLastError();
 }

@@ -55,15 +55,18 @@ cudaError_t scratch_for_current_device(void** out) {
 }  // namespace
 
 extern "C" mla_status mla_decode_static(const void* q, const void* cache, int64_t cap_blocks,
-                                        const int64_t* seq_block, const int32_t* kv_len, const void* W_UV, int B,
+                                        const int32_t* block_table, int max_blocks, const int32_t* kv_len,
+                                        const void* W_UV, int B,
                                         int n_q, int H, float scale, int num_splits, void* out, float* lse_out,
                                         int32_t* dev_status, mla_stream stream) {
     if (B < 0 || n_q < 1 || H < 1 || num_splits < 0) return MLA_ERR_INVALID_ARG;
     const size_t need = mla_decode_workspace_bytes(B, n_q, H, num_splits);
     if (need > static_cast<size_t>(MLA_DECODE_STATIC_SCRATCH_BYTES)) return MLA_ERR_WORKSPACE;
     if (B == 0) return MLA_OK;
+    // argument errors are reported before the device is touched, as for every other entry point
+    if (!q || !cache || !block_table || !kv_len || !W_UV || !out) return MLA_ERR_INVALID_ARG;
     void* scratch = nullptr;
     if (scratch_for_current_device(&scratch) != cudaSuccess) return MLA_ERR_CUDA;
-    return mla_decode(q, cache, cap_blocks, seq_block, kv_len, W_UV, B, n_q, H, scale, num_splits, scratch,
+    return mla_decode(q, cache, cap_blocks, block_table, max_blocks, kv_len, W_UV, B, n_q, H, scale, num_splits, scratch,
                       static_cast<size_t>(MLA_DECODE_STATIC_SCRATCH_BYTES), out, lse_out, dev_status, stream);
 }

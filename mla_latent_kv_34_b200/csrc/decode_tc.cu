@@ -43,6 +43,8 @@
 #include <cuda.h>
 #include <math_constants.h>
 
+#include <mutex>
+
 #include "mla_internal.cuh"
 #include "sm100.cuh"
 
@@ -112,30 +114,36 @@ static_assert(kMsgStride >= kMsgBytes, "message slot");
 
 struct Params {
     const uint16_t* q;
-    const uint8_t* cache;  // blocks of kBlockBytes
-    const int64_t* seq_block;
+    const uint8_t* cache;        // pool of blocks of kBlockBytes
+    const int32_t* block_table;  // [B][max_blocks] pool block of each 128-token tile of a sequence
     const int32_t* kv_len;
     float* o_part;    // [G][slots][128 column groups of 4][128 rows] x float4 (unnormalised O)
     float2* ml_part;  // [G][slots][128]  (running max in log2 units, sum)
     int32_t* dev_status;
     int64_t cap_blocks;
+    int max_blocks;
     int B, n_q, H, R, G, P_g, slots;
     float scale_log2;
 };
 
 __device__ __forceinline__ int seq_tiles(const Params& p, int b) {
-    const int L = p.kv_len[b];
-    if (L < p.n_q) return 0;
-    const int64_t s = p.seq_block[b];
-    const int nt = (L + kTile - 1) / kTile;
-    if (s < 0 || s + nt > p.cap_blocks) return 0;
-    return nt;
+    return valid_seq_tiles(p.kv_len[b], p.n_q, p.max_blocks);
 }
 
 struct Seg {
     int b, t0, t1, L, slot;
-    int64_t blk0;  // first cache block of the sequence
+    const int32_t* tab;  // the sequence's row of the block table
 };
+
+// Pool block of tile t of a segment; an entry outside the pool is reported and replaced by block 0
+// (that sequence's result is then unspecified, but no access leaves the pool).
+__device__ __forceinline__ const uint8_t* tile_src(const Params& p, int32_t e) {
+    if (e < 0 || e >= p.cap_blocks) {
+        if (p.dev_status) atomicOr(p.dev_status, MLA_DEVERR_ROW_RANGE);
+        e = 0;
+    }
+    return p.cache + static_cast<int64_t>(e) * kBlockBytes;
+}
 
 // Walks the segments of one cluster's tile range [lo, hi), starting at sequence b0 whose
 // first tile has global index tb0 (found once per CTA in the prologue).
@@ -160,7 +168,7 @@ struct SegWalk {
                 s.t0 = a - ctb;
                 s.t1 = e - ctb;
                 s.L = p.kv_len[cb];
-                s.blk0 = p.seq_block[cb];
+                s.tab = p.block_table + static_cast<int64_t>(cb) * p.max_blocks;
                 s.slot = cb + pidx;
                 return true;
             }
@@ -237,6 +245,10 @@ decode_tc_kernel(const Params p) {
         *resc_pb = 0;
         fence_mbar_init();
     }
+    if (warp == kWarpProducer) tmem_alloc(tmem_slot, 512);
+    // Everything above touches only this CTA's own resources, so it overlaps the previous kernel's tail
+    // under programmatic dependent launch; every read of the call's inputs comes after this wait.
+    grid_dependency_wait();
     if (warp == 0) {
         // total tiles, then (by a warp scan) the sequence holding this cluster's first tile
         int s = 0;
@@ -246,8 +258,7 @@ decode_tc_kernel(const Params p) {
             if (blockIdx.x == 0 && p.dev_status) {
                 const int L = p.kv_len[b];
                 if (L < p.n_q) atomicOr(p.dev_status, MLA_DEVERR_KV_LEN);
-                else if (p.seq_block[b] < 0 || p.seq_block[b] + (L + kTile - 1) / kTile > p.cap_blocks)
-                    atomicOr(p.dev_status, MLA_DEVERR_ROW_RANGE);
+                else if ((L + kTile - 1) / kTile > p.max_blocks) atomicOr(p.dev_status, MLA_DEVERR_ROW_RANGE);
             }
         }
 #pragma unroll
@@ -279,7 +290,6 @@ decode_tc_kernel(const Params p) {
             walk0[1] = tb0;
         }
     }
-    if (warp == kWarpProducer) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -311,7 +321,7 @@ decode_tc_kernel(const Params p) {
                 const uint64_t keep = l2_policy_evict_last();
                 while (ok && w.next(p, s)) {
                     for (int t = s.t0; ok && t < s.t1; ++t) {
-                        const uint8_t* src = p.cache + (s.blk0 + t) * kBlockBytes;
+                        const uint8_t* src = tile_src(p, s.tab[t]);
                         for (int k = 0; k < kCopies; ++k, ++nc) {
                             const uint32_t slot = nc % kRingSlots, u = nc / kRingSlots;
                             ok = mbar_wait(&bars[kSBarEmpty + slot], (u & 1u) ^ 1u, abort_flag, kLimitNs);
@@ -592,7 +602,7 @@ decode_tc_kernel(const Params p) {
                 const uint64_t last_use = l2_policy_evict_first();
                 while (ok && w.next(p, s)) {
                     for (int t = s.t0; ok && t < s.t1; ++t) {
-                        const uint8_t* src = p.cache + (s.blk0 + t) * kBlockBytes;
+                        const uint8_t* src = tile_src(p, s.tab[t]);
                         for (int k = 0; k < kVPerTile; ++k, ++nv) {
                             const uint32_t st = nv % kVStages, u = nv / kVStages;
                             if (!mbar_wait(&bars[kOBarVEmpty + st], (u & 1u) ^ 1u, abort_flag, kLimitNs)) {
@@ -784,6 +794,7 @@ decode_tc_kernel(const Params p) {
     }
 
     // ------------------------------------------------------------------ teardown
+    grid_dependents_launch();  // the merge kernel may be scheduled; it waits for this grid to finish
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // the peer no longer touches this CTA's shared memory
@@ -795,19 +806,20 @@ decode_tc_kernel(const Params p) {
 
 }  // namespace tc
 
-int decode_tc_max_clusters() { return 74; }
-
-// Co-resident clusters of the kernel on the current device (cached per device).
+// Co-resident clusters of the kernel on the current device, at most kMaxPairs (the workspace has a slot
+// per pair).  The occupancy query runs once per device; the table is guarded for concurrent callers.
 int decode_tc_clusters() {
+    static std::mutex mu;
     static int cache[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lock(mu);
     if (cache[dev] > 0) return cache[dev];
     if (cudaFuncSetAttribute(tc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::kSmemBytes) !=
         cudaSuccess)
         return 0;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * decode_tc_max_clusters());
+    cfg.gridDim = dim3(2 * kMaxPairs);
     cfg.blockDim = dim3(tc::kThreads);
     cfg.dynamicSmemBytes = tc::kSmemBytes;
     cudaLaunchAttribute attr[1];
@@ -819,13 +831,14 @@ int decode_tc_clusters() {
     cfg.numAttrs = 1;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, tc::decode_tc_kernel, &cfg) != cudaSuccess || n <= 0) return 0;
-    cache[dev] = n < decode_tc_max_clusters() ? n : decode_tc_max_clusters();
+    cache[dev] = n < kMaxPairs ? n : kMaxPairs;
     return cache[dev];
 }
 
-cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
-                             const int32_t* kv_len, int B, int n_q, int H, float scale, int clusters_per_group,
-                             float* o_part, float2* ml_part, int slots, int32_t* dev_status, cudaStream_t stream) {
+cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
+                             int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale,
+                             int clusters_per_group, float* o_part, float2* ml_part, int slots, int32_t* dev_status,
+                             cudaStream_t stream) {
     const int R = n_q * H;
     const int G = (R + tc::kRows - 1) / tc::kRows;
     int total = decode_tc_clusters();
@@ -840,12 +853,13 @@ cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t ca
     tc::Params prm;
     prm.q = q;
     prm.cache = cache;
-    prm.seq_block = seq_block;
+    prm.block_table = block_table;
     prm.kv_len = kv_len;
     prm.o_part = o_part;
     prm.ml_part = ml_part;
     prm.dev_status = dev_status;
     prm.cap_blocks = cap_blocks;
+    prm.max_blocks = max_blocks;
     prm.B = B;
     prm.n_q = n_q;
     prm.H = H;
@@ -859,13 +873,15 @@ cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t ca
     cfg.blockDim = dim3(tc::kThreads);
     cfg.dynamicSmemBytes = tc::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, tc::decode_tc_kernel, prm);
 }
 

@@ -35,20 +35,25 @@ DecodeWs decode_ws_layout(int B, int n_q, int H, int S) {
 mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
 // ---- tensor-core path: segment partials [G][slots][128 rows] float2 (m, l), then (1024-aligned)
-//      [G][slots] blocks of 128 rows x 512 fp32 O, each stored as [128 column groups of 4][128 rows] x float4
+//      [G][slots] blocks of 128 rows x 512 fp32 O, each stored as [128 column groups of 4][128 rows] x float4,
+//      then (1024-aligned) the merged latent output o_lat as bf16 operand tiles, [H][olat_rows(T)] x 1 KB.
+//      A slot per (sequence + CTA pair): a pair's tile range starts at most one piece into a sequence.
 struct TcWs {
     int G, slots;
-    size_t ml_part, o_part, total;
+    size_t ml_part, o_part, olat, total;
 };
+
+size_t align1k(size_t x) { return ((x + 1023) / 1024) * 1024; }
 
 TcWs tc_ws_layout(int B, int n_q, int H) {
     TcWs w;
     w.G = (n_q * H + 127) / 128;
-    w.slots = B + decode_tc_max_clusters();
+    w.slots = B + kMaxPairs;
     const size_t rows = static_cast<size_t>(w.G) * w.slots * 128;
     w.ml_part = 0;
-    w.o_part = ((rows * sizeof(float2) + 1023) / 1024) * 1024;
-    w.total = w.o_part + rows * kDc * sizeof(float);
+    w.o_part = align1k(rows * sizeof(float2));
+    w.olat = align1k(w.o_part + rows * kDc * sizeof(float));
+    w.total = w.olat + static_cast<size_t>(H) * olat_rows(B * n_q) * 1024;
     return w;
 }
 
@@ -61,10 +66,16 @@ int tc_clusters_per_group(int G, int num_splits) {
     return pg;
 }
 
-mla_status check_decode_shape(int B, int64_t cap_blocks, int n_q, int H, int num_splits) {
-    if (B < 0 || cap_blocks < 0 || cap_blocks >= (int64_t(1) << 31) / kBlockTokens) return MLA_ERR_INVALID_ARG;
+constexpr int64_t kMaxPoolBlocks = 0x7FFFFFFF;                 // block-table entries are int32
+constexpr int kMaxTableBlocks = 0x7FFFFFFF / kBlockTokens;      // positions are int32
+
+mla_status check_decode_shape(int B, int64_t cap_blocks, int max_blocks, int n_q, int H, int num_splits) {
+    if (B < 0 || cap_blocks < 0 || cap_blocks > kMaxPoolBlocks || max_blocks < 0 || max_blocks > kMaxTableBlocks)
+        return MLA_ERR_INVALID_ARG;
+    if (B > 0 && (cap_blocks < 1 || max_blocks < 1)) return MLA_ERR_INVALID_ARG;
     if (H < 1 || H > kMaxHeads || n_q < 1 || n_q > kMaxNq || num_splits < 0 || num_splits > 256)
         return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<int64_t>(B) * n_q > 0x7FFFFFFF / kMaxHeads) return MLA_ERR_UNSUPPORTED_SHAPE;
     return MLA_OK;
 }
 
@@ -72,13 +83,14 @@ mla_status check_decode_shape(int B, int64_t cap_blocks, int n_q, int H, int num
 
 extern "C" {
 
-int mla_abi_version(void) { return 1; }
+int mla_abi_version(void) { return 2; }
 
 const char* mla_status_string(int status) {
     switch (status) {
         case MLA_OK: return "ok";
         case MLA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, negative or too large size)";
-        case MLA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (H in 1..128, n_q in 1..16, splits in 0..256)";
+        case MLA_ERR_UNSUPPORTED_SHAPE:
+            return "unsupported shape (H in 1..128, n_q in 1..16, splits in 0..256, B * n_q * 128 < 2^31)";
         case MLA_ERR_CUDA: return "CUDA runtime error";
         case MLA_ERR_WORKSPACE: return "workspace too small";
         default: return "unknown status";
@@ -135,17 +147,22 @@ mla_status mla_query_up(const void* c_q, const void* W_UQ, const void* W_QR, int
                                        static_cast<uint16_t*>(q_rope), dev_status, static_cast<cudaStream_t>(stream)));
 }
 
-mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int64_t* seq_block, const int32_t* seq_idx,
-                            const int32_t* pos, const void* c_kv, const void* k_rope, const float* rope_table,
-                            int64_t rope_len, int T, int32_t* dev_status, mla_stream stream) {
-    if (T < 0 || cap_blocks < 0 || rope_len < 0) return MLA_ERR_INVALID_ARG;
+mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int32_t* block_table, int num_seqs,
+                            int max_blocks, const int32_t* seq_idx, const int32_t* pos, const void* c_kv, const void* k_rope,
+                            const float* rope_table, int64_t rope_len, int T, int32_t* dev_status,
+                            mla_stream stream) {
+    if (T < 0 || cap_blocks < 0 || cap_blocks > kMaxPoolBlocks || rope_len < 0 || max_blocks < 0 || num_seqs < 0)
+        return MLA_ERR_INVALID_ARG;
     if (T == 0) return MLA_OK;
-    if (!cache || !seq_block || !seq_idx || !pos || !c_kv || !k_rope || !rope_table) return MLA_ERR_INVALID_ARG;
+    if (!cache || !block_table || !seq_idx || !pos || !c_kv || !k_rope || !rope_table || max_blocks < 1 ||
+        num_seqs < 1)
+        return MLA_ERR_INVALID_ARG;
     if (!aligned16(cache) || !aligned16(c_kv) || !aligned16(k_rope) || !aligned16(rope_table))
         return MLA_ERR_INVALID_ARG;
-    return cuda_status(launch_append_cache(static_cast<uint8_t*>(cache), cap_blocks, seq_block, seq_idx, pos,
-                                           static_cast<const uint16_t*>(c_kv), static_cast<const uint16_t*>(k_rope),
-                                           rope_table, rope_len, T, dev_status, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_append_cache(static_cast<uint8_t*>(cache), cap_blocks, block_table, num_seqs,
+                                           max_blocks, seq_idx, pos, static_cast<const uint16_t*>(c_kv),
+                                           static_cast<const uint16_t*>(k_rope), rope_table, rope_len, T, dev_status,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits) {
@@ -153,14 +170,15 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits) {
     return tc_ws_layout(B, n_q, H).total;
 }
 
-mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_blocks, const int64_t* seq_block,
-                             const int32_t* kv_len, int B, int n_q, int H, float scale, int num_splits,
-                             void* workspace, size_t ws_bytes, int32_t* dev_status, mla_stream stream) {
-    mla_status st = check_decode_shape(B, cap_blocks, n_q, H, num_splits);
+mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_blocks, const int32_t* block_table,
+                             int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale,
+                             int num_splits, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                             mla_stream stream) {
+    mla_status st = check_decode_shape(B, cap_blocks, max_blocks, n_q, H, num_splits);
     if (st != MLA_OK) return st;
     if (!(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
     if (B == 0) return MLA_OK;
-    if (!q || !cache || !seq_block || !kv_len || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!q || !cache || !block_table || !kv_len || !workspace) return MLA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(cache) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
     const TcWs lay = tc_ws_layout(B, n_q, H);
     if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
@@ -168,43 +186,46 @@ mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_block
     if (pg <= 0) return MLA_ERR_CUDA;
     char* ws = static_cast<char*>(workspace);
     return cuda_status(launch_decode_tc(static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(cache),
-                                        cap_blocks, seq_block, kv_len, B, n_q, H, scale, pg,
+                                        cap_blocks, block_table, max_blocks, kv_len, B, n_q, H, scale, pg,
                                         reinterpret_cast<float*>(ws + lay.o_part),
                                         reinterpret_cast<float2*>(ws + lay.ml_part), lay.slots, dev_status,
                                         static_cast<cudaStream_t>(stream)));
 }
 
-mla_status mla_decode_finish(const int64_t* seq_block, const int32_t* kv_len, int64_t cap_blocks, const void* W_UV,
-                             int B, int n_q, int H, int num_splits, void* workspace, size_t ws_bytes, void* out,
-                             float* lse_out, int32_t* dev_status, mla_stream stream) {
-    mla_status st = check_decode_shape(B, cap_blocks, n_q, H, num_splits);
+mla_status mla_decode_finish(const int32_t* kv_len, int max_blocks, const void* W_UV, int B, int n_q, int H,
+                             int num_splits, void* workspace, size_t ws_bytes, void* out, float* lse_out,
+                             int32_t* dev_status, mla_stream stream) {
+    mla_status st = check_decode_shape(B, B > 0 ? 1 : 0, max_blocks, n_q, H, num_splits);
     if (st != MLA_OK) return st;
     if (B == 0) return MLA_OK;
-    if (!seq_block || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
     if (!aligned16(W_UV) || !aligned16(out) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
     const TcWs lay = tc_ws_layout(B, n_q, H);
     if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
     const int pg = tc_clusters_per_group(lay.G, num_splits);
     if (pg <= 0) return MLA_ERR_CUDA;
-    const char* ws = static_cast<const char*>(workspace);
-    return cuda_status(launch_finish_tc(reinterpret_cast<const float*>(ws + lay.o_part),
-                                        reinterpret_cast<const float2*>(ws + lay.ml_part), kv_len, seq_block,
-                                        cap_blocks, B, n_q, H, pg, lay.slots, static_cast<const uint16_t*>(W_UV),
-                                        static_cast<uint16_t*>(out), lse_out, dev_status,
-                                        static_cast<cudaStream_t>(stream)));
+    char* ws = static_cast<char*>(workspace);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_merge(reinterpret_cast<const float*>(ws + lay.o_part),
+                                 reinterpret_cast<const float2*>(ws + lay.ml_part), kv_len, max_blocks, B, n_q, H, pg,
+                                 lay.slots, reinterpret_cast<uint8_t*>(ws + lay.olat), lse_out, dev_status, cs);
+    if (e != cudaSuccess) return MLA_ERR_CUDA;
+    return cuda_status(launch_upproj(reinterpret_cast<const uint8_t*>(ws + lay.olat),
+                                     static_cast<const uint16_t*>(W_UV), B * n_q, H, static_cast<uint16_t*>(out),
+                                     dev_status, cs));
 }
 
-mla_status mla_decode(const void* q, const void* cache, int64_t cap_blocks, const int64_t* seq_block,
+mla_status mla_decode(const void* q, const void* cache, int64_t cap_blocks, const int32_t* block_table, int max_blocks,
                       const int32_t* kv_len, const void* W_UV, int B, int n_q, int H, float scale, int num_splits,
                       void* workspace, size_t ws_bytes, void* out, float* lse_out, int32_t* dev_status,
                       mla_stream stream) {
     if (B > 0 && (!W_UV || !out)) return MLA_ERR_INVALID_ARG;
     if (B > 0 && (!aligned16(W_UV) || !aligned16(out))) return MLA_ERR_INVALID_ARG;
-    mla_status st = mla_decode_attend(q, cache, cap_blocks, seq_block, kv_len, B, n_q, H, scale, num_splits,
-                                      workspace, ws_bytes, dev_status, stream);
+    mla_status st = mla_decode_attend(q, cache, cap_blocks, block_table, max_blocks, kv_len, B, n_q, H, scale,
+                                      num_splits, workspace, ws_bytes, dev_status, stream);
     if (st != MLA_OK || B == 0) return st;
-    return mla_decode_finish(seq_block, kv_len, cap_blocks, W_UV, B, n_q, H, num_splits, workspace, ws_bytes, out,
-                             lse_out, dev_status, stream);
+    return mla_decode_finish(kv_len, max_blocks, W_UV, B, n_q, H, num_splits, workspace, ws_bytes, out, lse_out,
+                             dev_status, stream);
 }
 
 size_t mla_decode_cudacore_workspace_bytes(int B, int n_q, int H, int num_splits) {
@@ -213,15 +234,15 @@ size_t mla_decode_cudacore_workspace_bytes(int B, int n_q, int H, int num_splits
     return decode_ws_layout(B, n_q, H, S).total;
 }
 
-mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_blocks, const int64_t* seq_block,
-                               const int32_t* kv_len, const void* W_UV, int B, int n_q, int H, float scale,
-                               int num_splits, void* workspace, size_t ws_bytes, void* out, float* lse_out,
-                               int32_t* dev_status, mla_stream stream) {
-    mla_status st = check_decode_shape(B, cap_blocks, n_q, H, num_splits);
+mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_blocks, const int32_t* block_table,
+                               int max_blocks, const int32_t* kv_len, const void* W_UV, int B, int n_q, int H,
+                               float scale, int num_splits, void* workspace, size_t ws_bytes, void* out,
+                               float* lse_out, int32_t* dev_status, mla_stream stream) {
+    mla_status st = check_decode_shape(B, cap_blocks, max_blocks, n_q, H, num_splits);
     if (st != MLA_OK) return st;
     if (!(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
     if (B == 0) return MLA_OK;
-    if (!q || !cache || !seq_block || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!q || !cache || !block_table || !kv_len || !W_UV || !out || !workspace) return MLA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(cache) || !aligned16(W_UV) || !aligned16(out) || !aligned16(workspace))
         return MLA_ERR_INVALID_ARG;
     const int S = num_splits ? num_splits : auto_splits(B, n_q, H);
@@ -231,8 +252,8 @@ mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_blo
     float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + lay.lse_part);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_decode_simt(static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(cache),
-                                       cap_blocks, seq_block, kv_len, B, n_q, H, scale, S, o_part, lse_part,
-                                       dev_status, cs);
+                                       cap_blocks, block_table, max_blocks, kv_len, B, n_q, H, scale, S, o_part,
+                                       lse_part, dev_status, cs);
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     return cuda_status(launch_combine(o_part, lse_part, B * n_q, H, S, static_cast<const uint16_t*>(W_UV), out,
                                       lse_out, cs));

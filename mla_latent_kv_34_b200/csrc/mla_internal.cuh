@@ -19,6 +19,16 @@ constexpr int kBlockTokens = MLA_BLOCK_TOKENS;  // tokens per cache block
 constexpr int kBlockBytes = MLA_BLOCK_BYTES;    // 9 chunks x [128 rows x 128 B]
 constexpr int kBlockChunk = kBlockTokens * 128;  // bytes of one 64-column chunk of a block
 static_assert(kBlockBytes == 9 * kBlockChunk, "block layout");
+constexpr int kMaxPairs = 74;      // CTA pairs per row group the tensor-core decode uses at most (148 SMs / 2)
+
+// Tiles (128-token blocks) of a sequence that the decode processes: none when kv_len < n_q or when the
+// sequence needs more blocks than its block-table row holds.  The attend and merge kernels both use this
+// rule, so they agree on how the (sequence, tile) space is cut into pieces.
+__host__ __device__ __forceinline__ int valid_seq_tiles(int L, int n_q, int max_blocks) {
+    if (L < n_q) return 0;
+    const int nt = (L + kBlockTokens - 1) / kBlockTokens;
+    return nt > max_blocks ? 0 : nt;
+}
 
 // Byte offset of column c of row r inside a cache block (128-byte swizzle per 64-column chunk).
 __host__ __device__ __forceinline__ int block_offset(int r, int c) {
@@ -46,10 +56,11 @@ __device__ __forceinline__ void report(int32_t* dev_status, int32_t bit) {
 }
 
 // Host-side launch wrappers (one per kernel file).
-cudaError_t launch_append_cache(uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block, const int32_t* seq_idx,
-                                const int32_t* pos, const uint16_t* c_kv, const uint16_t* k_rope,
-                                const float* rope_table, int64_t rope_len, int T, int32_t* dev_status,
-                                cudaStream_t stream);
+cudaError_t launch_append_cache(uint8_t* cache, int64_t cap_blocks, const int32_t* block_table, int num_seqs,
+                                int max_blocks,
+                                const int32_t* seq_idx, const int32_t* pos, const uint16_t* c_kv,
+                                const uint16_t* k_rope, const float* rope_table, int64_t rope_len, int T,
+                                int32_t* dev_status, cudaStream_t stream);
 
 cudaError_t launch_absorb_tc(const uint16_t* q_nope, const uint16_t* q_rope, const int32_t* pos, const uint16_t* W_UK,
                              const float* rope_table, int64_t rope_len, int T, int H, uint16_t* q_out,
@@ -59,21 +70,29 @@ cudaError_t launch_absorb_tc(const uint16_t* q_nope, const uint16_t* q_rope, con
 cudaError_t launch_query_up(const uint16_t* c_q, const uint16_t* W_UQ, const uint16_t* W_QR, int T, int H, int d_cq,
                             uint16_t* q_nope, uint16_t* q_rope, int32_t* dev_status, cudaStream_t stream);
 
-cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
-                               const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,
+cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
+                               int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,
                                float* o_part, float* lse_part, int32_t* dev_status, cudaStream_t stream);
 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int T, int H, int splits,
                            const uint16_t* W_UV, void* out, float* lse_out, cudaStream_t stream);
 
-// Tensor-core decode (decode_tc.cu); projections and the merge of its segments (proj_tc.cu).
-int decode_tc_max_clusters();
+// Tensor-core decode (decode_tc.cu); the merge of its pieces and the W^UV projection (proj_tc.cu).
 int decode_tc_clusters();
-cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int64_t* seq_block,
-                             const int32_t* kv_len, int B, int n_q, int H, float scale, int clusters_per_group,
-                             float* o_part, float2* ml_part, int slots, int32_t* dev_status, cudaStream_t stream);
-cudaError_t launch_finish_tc(const float* o_part, const float2* ml_part, const int32_t* kv_len, const int64_t* seq_block,
-                             int64_t cap_blocks, int B, int n_q, int H, int P_g, int slots, const uint16_t* W_UV,
-                             uint16_t* out, float* lse_out, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
+                             int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale,
+                             int clusters_per_group, float* o_part, float2* ml_part, int slots, int32_t* dev_status,
+                             cudaStream_t stream);
+// Rows of the merged latent output o_lat kept for the up-projection: T rounded so that every 64-token
+// block but the last is full and the last is a multiple of 16 (the MMA N granularity).
+__host__ __device__ __forceinline__ int olat_rows(int T) {
+    const int full = (T / 64) * 64, rest = T - full;
+    return full + ((rest + 15) / 16) * 16;
+}
+cudaError_t launch_merge(const float* o_part, const float2* ml_part, const int32_t* kv_len, int max_blocks, int B,
+                         int n_q, int H, int P_g, int slots, uint8_t* olat, float* lse_out, int32_t* dev_status,
+                         cudaStream_t stream);
+cudaError_t launch_upproj(const uint8_t* olat, const uint16_t* W_UV, int T, int H, uint16_t* out, int32_t* dev_status,
+                          cudaStream_t stream);
 
 }  // namespace mla

@@ -37,6 +37,17 @@ __device__ __forceinline__ uint32_t mapa(uint32_t local_smem_addr, uint32_t rank
     return r;
 }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+
+// Wait until every grid this one depends on (the previous kernel on the stream, when this grid was
+// launched with programmatic stream serialization) has completed and its memory is visible.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next grid on the stream be scheduled before this one ends (it still waits for this grid's
+// completion in its own grid_dependency_wait before reading what this grid wrote).
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -58,9 +58,9 @@ def rel_l2(got: np.ndarray, ref: np.ndarray) -> float:
 class Problem:
     cfg: mi.MLAConfig
     lengths: np.ndarray
-    starts: np.ndarray  # first block of each sequence
+    tables: np.ndarray  # int32 [B, max_blocks] pool block of each tile of each sequence
     cache: torch.Tensor
-    seq_block: torch.Tensor
+    block_table: torch.Tensor
     kv_len: torch.Tensor
     q_nope: torch.Tensor
     q_rope: torch.Tensor
@@ -80,7 +80,7 @@ class Problem:
     def decode(self, q, num_splits=0, lse=True, path="tc"):
         lse_out = torch.empty((self.T, self.cfg.H), dtype=torch.float32, device=q.device) if lse else None
         fn = mla.decode if path == "tc" else mla.decode_cudacore
-        out = fn(q, self.cache, self.seq_block, self.kv_len, self.W_UV, self.cfg.n_q, self.cfg.scale,
+        out = fn(q, self.cache, self.block_table, self.kv_len, self.W_UV, self.cfg.n_q, self.cfg.scale,
                  num_splits=num_splits, lse_out=lse_out, dev_status=self.status)
         return out, lse_out
 
@@ -94,39 +94,75 @@ class Problem:
                                self.cfg.n_q, scale=self.cfg.scale, base=self.cfg.rope_base, heads=heads)
 
 
-def build_problem(cfg: mi.MLAConfig, lengths=None, slack_blocks: int = 2, dev="cuda",
-                  chunk_rows: int = 1 << 16, gap_blocks: int = 0) -> Problem:
-    """Fill a blocked cache with every sequence's tokens via mla_append_cache.
+def block_tables(lengths, gap_blocks: int = 0, slack_blocks: int = 2, shuffle_seed=None, extra_cols: int = 0):
+    """Block tables of a pool holding every sequence: (tables int32 [B, max_blocks], cap_blocks, unowned blocks).
 
-    Sequences occupy consecutive blocks from block 0 (``gap_blocks`` apart);
-    every byte not written by an append (the tails of last blocks, the gaps and
-    ``slack_blocks`` extra blocks) holds the bf16 NaN pattern, so a kernel that
-    used a row outside a sequence would be noticed.
+    Contiguous (default): sequences take consecutive blocks from block 0, ``gap_blocks`` apart, with
+    ``slack_blocks`` spare blocks at the end.  Shuffled (``shuffle_seed``): every block of the pool,
+    including about one unowned block per sequence, is placed by a seeded random permutation, so the
+    blocks of a sequence are scattered and out of order.  ``extra_cols`` adds table columns past the
+    longest sequence.  Every entry past a sequence's own blocks names an unowned block.
+    """
+    lengths = np.asarray(lengths, dtype=np.int64)
+    B = len(lengths)
+    nblk = (lengths + BLOCK_TOKENS - 1) // BLOCK_TOKENS
+    max_blocks = int(nblk.max()) + extra_cols
+    if shuffle_seed is None:
+        starts = np.zeros(B, dtype=np.int64)
+        if B > 1:
+            starts[1:] = np.cumsum(nblk[:-1] + gap_blocks)
+        cap = int(starts[-1] + nblk[-1]) + slack_blocks
+        owned = np.zeros(cap, dtype=bool)
+        tables = np.zeros((B, max_blocks), dtype=np.int32)
+        for b in range(B):
+            tables[b, :nblk[b]] = starts[b] + np.arange(nblk[b])
+            owned[starts[b]:starts[b] + nblk[b]] = True
+    else:
+        cap = int(nblk.sum()) + B + slack_blocks
+        perm = np.random.default_rng(shuffle_seed).permutation(cap).astype(np.int32)
+        tables = np.zeros((B, max_blocks), dtype=np.int32)
+        owned = np.zeros(cap, dtype=bool)
+        k = 0
+        for b in range(B):
+            tables[b, :nblk[b]] = perm[k:k + nblk[b]]
+            owned[perm[k:k + nblk[b]]] = True
+            k += int(nblk[b])
+    unowned = np.flatnonzero(~owned)
+    assert len(unowned) > 0
+    for b in range(B):
+        n = max_blocks - int(nblk[b])
+        tables[b, nblk[b]:] = unowned[np.arange(n) % len(unowned)]
+    return tables, cap, unowned
+
+
+def build_problem(cfg: mi.MLAConfig, lengths=None, slack_blocks: int = 2, dev="cuda",
+                  chunk_rows: int = 1 << 16, gap_blocks: int = 0, shuffle_seed=None, extra_cols: int = 0) -> Problem:
+    """Fill a paged cache with every sequence's tokens via mla_append_cache.
+
+    Block tables come from ``block_tables`` (contiguous or shuffled).  Every byte not written by an
+    append (the tails of last blocks and all unowned blocks) holds the bf16 NaN pattern, so a kernel
+    that used a row outside a sequence, or a table entry past a sequence's blocks, would be noticed.
     """
     lengths = mi.kv_lengths(cfg) if lengths is None else np.asarray(lengths, dtype=np.int64)
     pool_starts = mi.seq_starts(lengths)            # rows in the generator's packed pool
-    nblk = (lengths + BLOCK_TOKENS - 1) // BLOCK_TOKENS
-    seq_block = np.zeros(cfg.B, dtype=np.int64)
-    if cfg.B > 1:
-        seq_block[1:] = np.cumsum(nblk[:-1] + gap_blocks)
-    cap_blocks = int(seq_block[-1] + nblk[-1]) + slack_blocks
+    tables, cap_blocks, _ = block_tables(lengths, gap_blocks, slack_blocks, shuffle_seed, extra_cols)
     N = int(lengths.sum())
     cache = torch.full((cap_blocks, BLOCK_BYTES // 2), NAN_BF16, dtype=torch.int16, device=dev).view(torch.uint8)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     rope_tab = mla.rope_table(int(lengths.max()), cfg.rope_base, dev)
-    seq_block_t = torch.from_numpy(seq_block).to(dev)
+    table_t = torch.from_numpy(tables).to(dev)
     # per-row (sequence, position) of the whole pool
     seq_of_row = np.repeat(np.arange(cfg.B, dtype=np.int32), lengths)
     pos_of_row = (np.arange(N, dtype=np.int64) - np.repeat(pool_starts, lengths)).astype(np.int32)
     for r0 in range(0, N, chunk_rows):
         n = min(chunk_rows, N - r0)
         c, k = mi.token_rows(cfg, r0, n)
-        mla.append_cache(cache, seq_block_t, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
+        mla.append_cache(cache, table_t, torch.from_numpy(seq_of_row[r0:r0 + n]).to(dev),
                          torch.from_numpy(pos_of_row[r0:r0 + n]).to(dev), to_dev_bf16(c, dev),
                          to_dev_bf16(k, dev), rope_tab, status)
     qn, qr = mi.queries(cfg)
     q_pos = np.concatenate([lengths[b] - cfg.n_q + np.arange(cfg.n_q) for b in range(cfg.B)]).astype(np.int32)
-    return Problem(cfg, lengths, seq_block, cache, seq_block_t,
+    return Problem(cfg, lengths, tables, cache, table_t,
                    torch.from_numpy(lengths.astype(np.int32)).to(dev),
                    to_dev_bf16(qn, dev), to_dev_bf16(qr, dev), torch.from_numpy(q_pos).to(dev),
                    to_dev_bf16(mi.weights(cfg, "uk"), dev), to_dev_bf16(mi.weights(cfg, "uv"), dev),

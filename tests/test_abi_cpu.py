@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol(mla):
     for n in names:
         assert hasattr(mla.lib, n), n
     assert set(names) == set(mla.EXPORTED)
-    assert mla.lib.mla_abi_version() == 1
+    assert mla.lib.mla_abi_version() == 2
 
 
 def test_rope_table_matches_oracle_bitwise(mla):
@@ -56,26 +56,38 @@ def test_host_validation_rejects_bad_arguments(mla):
     L = mla.lib
     fake = ctypes.c_void_p(4096)  # never dereferenced: validation fails first
     odd = ctypes.c_void_p(4098)
-    # decode: null q, unsupported H / n_q / splits, bad scale, small workspace
-    assert L.mla_decode(None, fake, 10, fake, fake, fake, 1, 1, 16, 0.07, 0, fake, 1 << 30, fake, None, None, None) == 1
-    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 1, 1, 129, 0.07, 0, fake, 1 << 30, fake, None, None, None) == 2
-    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 1, 0, 16, 0.07, 0, fake, 1 << 30, fake, None, None, None) == 2
-    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 1, 1, 16, 0.07, 300, fake, 1 << 30, fake, None, None, None) == 2
-    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 1, 1, 16, -1.0, 0, fake, 1 << 30, fake, None, None, None) == 1
-    assert L.mla_decode(odd, fake, 10, fake, fake, fake, 1, 1, 16, 0.07, 0, fake, 1 << 30, fake, None, None, None) == 1
+    # decode: null q, unsupported H / n_q / splits, bad scale, small workspace, bad pool / table sizes
+    def dec(q=fake, cap=10, mb=4, B=1, n_q=1, H=16, scale=0.07, splits=0, ws_bytes=1 << 30):
+        return L.mla_decode(q, fake, cap, fake, mb, fake, fake, B, n_q, H, scale, splits, fake, ws_bytes, fake, None,
+                            None, None)
+    assert dec(q=None) == 1
+    assert dec(H=129) == 2
+    assert dec(n_q=0) == 2
+    assert dec(splits=300) == 2
+    assert dec(scale=-1.0) == 1
+    assert dec(q=odd) == 1
+    assert dec(cap=0) == 1
+    assert dec(mb=0) == 1
+    assert dec(cap=1 << 31) == 1
     need = L.mla_decode_workspace_bytes(4, 2, 128, 3)
     assert need > 0
-    assert L.mla_decode(fake, fake, 10, fake, fake, fake, 4, 2, 128, 0.07, 3, fake, need - 1, fake, None, None,
-                        None) == 4
+    assert dec(B=4, n_q=2, H=128, splits=3, ws_bytes=need - 1) == 4
     # empty batch is a no-op
-    assert L.mla_decode(None, None, 0, None, None, None, 0, 1, 16, 0.07, 0, None, 0, None, None, None, None) == 0
+    assert L.mla_decode(None, None, 0, None, 0, None, None, 0, 1, 16, 0.07, 0, None, 0, None, None, None, None) == 0
+    # the two phases validate the same way
+    assert L.mla_decode_attend(fake, fake, 10, fake, 0, fake, 1, 1, 16, 0.07, 0, fake, 1 << 30, None, None) == 1
+    assert L.mla_decode_finish(fake, 0, fake, 1, 1, 16, 0, fake, 1 << 30, fake, None, None, None) == 1
+    assert L.mla_decode_finish(None, 4, fake, 1, 1, 16, 0, fake, 1 << 30, fake, None, None, None) == 1
     # absorb / append / combine
     assert L.mla_absorb_q(fake, fake, None, fake, None, 0, 4, 0, fake, None, None) == 2
     assert L.mla_absorb_q(None, fake, None, fake, None, 0, 4, 16, fake, None, None) == 1
     assert L.mla_absorb_q(None, None, None, None, None, 0, 0, 16, None, None, None) == 0
-    assert L.mla_append_cache(fake, 10, fake, fake, fake, fake, fake, None, 5, 3, None, None) == 1
-    assert L.mla_append_cache(fake, -1, fake, fake, fake, fake, fake, fake, 5, 3, None, None) == 1
-    assert L.mla_append_cache(None, 0, None, None, None, None, None, None, 0, 0, None, None) == 0
+    assert L.mla_append_cache(fake, 10, fake, 2, 4, fake, fake, fake, fake, None, 5, 3, None, None) == 1
+    assert L.mla_append_cache(fake, -1, fake, 2, 4, fake, fake, fake, fake, fake, 5, 3, None, None) == 1
+    assert L.mla_append_cache(fake, 10, fake, 2, 0, fake, fake, fake, fake, fake, 5, 3, None, None) == 1
+    assert L.mla_append_cache(fake, 10, fake, 0, 4, fake, fake, fake, fake, fake, 5, 3, None, None) == 1
+    assert L.mla_append_cache(fake, 10, None, 2, 4, fake, fake, fake, fake, fake, 5, 3, None, None) == 1
+    assert L.mla_append_cache(None, 0, None, 0, 0, None, None, None, None, None, 0, 0, None, None) == 0
     assert L.mla_splitkv_combine(fake, fake, 4, 16, 0, None, fake, None, None) == 2
     assert L.mla_splitkv_combine(None, fake, 4, 16, 2, None, fake, None, None) == 1
     # query up-projection: empty, d_cq not a multiple of 64, no heads, null input
@@ -87,10 +99,21 @@ def test_host_validation_rejects_bad_arguments(mla):
 
 
 def test_workspace_sizes(mla):
-    # tensor-core path: one slot per (sequence + CTA pair) and row group, any split count
+    # tensor-core path: one slot per (sequence + CTA pair) and row group, any split count, plus the merged
+    # latent output (bf16, rows rounded to 64-row blocks with a last block of a multiple of 16)
     a = mla.decode_workspace_bytes(32, 1, 128, 1)
     assert a == mla.decode_workspace_bytes(32, 1, 128, 0) > 32 * 128 * 512 * 4
     assert mla.decode_workspace_bytes(32, 2, 128, 0) > 1.9 * a
+    slot = 128 * (8 + 512 * 4)
+    for B, n_q, H in [(32, 1, 128), (128, 2, 128), (1, 1, 16), (70, 1, 3)]:
+        G = (n_q * H + 127) // 128
+        rows = G * (B + 74) * 128
+        T = B * n_q
+        olat_rows = (T // 64) * 64 + ((T % 64 + 15) // 16) * 16
+        head = -(-rows * 8 // 1024) * 1024
+        want = -(-(head + rows * 512 * 4) // 1024) * 1024 + H * olat_rows * 1024
+        assert mla.decode_workspace_bytes(B, n_q, H, 0) == want, (B, n_q, H)
+        assert want >= rows * slot // 128
     # CUDA-core path: one fp32 partial per split
     c1 = mla.lib.mla_decode_cudacore_workspace_bytes(32, 1, 128, 1)
     c4 = mla.lib.mla_decode_cudacore_workspace_bytes(32, 1, 128, 4)

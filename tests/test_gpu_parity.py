@@ -50,14 +50,16 @@ def _check_decode(prob, out, lse, seqs, heads=None, label=""):
 # ----------------------------------------------------------------- append
 
 def test_append_bit_exact_with_canary(cuda_ok, H):
-    """Appended rows equal the fp32 emulation bit for bit; no other byte changes."""
+    """Appended rows equal the fp32 emulation bit for bit, in the pool blocks a shuffled block table names;
+    no other byte changes."""
     dev = "cuda"
     import mla_latent_kv_34_b200 as mla
     cap_blocks = 80
     canary = np.full((cap_blocks, H.BLOCK_BYTES // 2), 0xA5A5, dtype=np.uint16)
     cache = torch.from_numpy(canary.view(np.int16).copy()).to(dev).view(torch.uint8)
-    seq_block = np.array([0, 17, 40, 63], dtype=np.int64)
     rng = np.random.default_rng(1)
+    # 4 sequences x 8 blocks scattered over the 80-block pool, in no order
+    tables = rng.permutation(cap_blocks)[:32].astype(np.int32).reshape(4, 8)
     T = 777
     seq_idx = rng.integers(0, 4, T).astype(np.int32)
     # distinct positions per sequence so no row is written twice
@@ -69,14 +71,14 @@ def test_append_bit_exact_with_canary(cuda_ok, H):
     k = mi.normal_bf16(77, 2, 0, T * 64).reshape(T, 64)
     tab = mla.rope_table(1000, 10000.0, dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    mla.append_cache(cache, torch.from_numpy(seq_block).to(dev), torch.from_numpy(seq_idx).to(dev),
+    mla.append_cache(cache, torch.from_numpy(tables).to(dev), torch.from_numpy(seq_idx).to(dev),
                      torch.from_numpy(pos).to(dev), H.to_dev_bf16(c, dev), H.to_dev_bf16(k, dev), tab, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     # logical rows from the oracle's fp32 emulation, placed per the documented block layout
     rows = np.concatenate([c, oapp.rotate_k_bits(k, pos)], axis=1)
     expect = canary.copy()
-    blk = seq_block[seq_idx] + pos // H.BLOCK_TOKENS
+    blk = tables[seq_idx, pos // H.BLOCK_TOKENS]
     H.pack_rows(expect, blk, pos % H.BLOCK_TOKENS, rows)
     got = H.cache_u16(cache)
     np.testing.assert_array_equal(H.unpack_rows(got, blk, pos % H.BLOCK_TOKENS), rows)
@@ -94,9 +96,11 @@ def test_append_large_positions_bit_exact(cuda_ok, H):
     k = mi.normal_bf16(78, 2, 0, T * 64).reshape(T, 64)
     tab = mla.rope_table(131072, 10000.0, dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    mla.append_cache(cache, torch.zeros(1, dtype=torch.int64, device=dev), torch.zeros(T, dtype=torch.int32, device=dev),
+    table = torch.arange(cap_blocks, dtype=torch.int32, device=dev).flip(0).reshape(1, cap_blocks)
+    mla.append_cache(cache, table, torch.zeros(T, dtype=torch.int32, device=dev),
                      torch.from_numpy(pos).to(dev), H.to_dev_bf16(c, dev), H.to_dev_bf16(k, dev), tab, st)
-    got = H.unpack_rows(H.cache_u16(cache), pos // H.BLOCK_TOKENS, pos % H.BLOCK_TOKENS)
+    blk = cap_blocks - 1 - pos // H.BLOCK_TOKENS
+    got = H.unpack_rows(H.cache_u16(cache), blk, pos % H.BLOCK_TOKENS)
     np.testing.assert_array_equal(got[:, :512], c)
     np.testing.assert_array_equal(got[:, 512:], oapp.rotate_k_bits(k, pos))
     assert int(st.item()) == 0
@@ -107,19 +111,26 @@ def test_append_out_of_range_is_reported_and_skipped(cuda_ok, H):
     dev = "cuda"
     cache = torch.zeros((3, H.BLOCK_BYTES), dtype=torch.uint8, device=dev)
     tab = mla.rope_table(256, 10000.0, dev)
-    c = torch.ones((2, 512), dtype=torch.bfloat16, device=dev)
-    k = torch.ones((2, 64), dtype=torch.bfloat16, device=dev)
+    c = torch.ones((3, 512), dtype=torch.bfloat16, device=dev)
+    k = torch.ones((3, 64), dtype=torch.bfloat16, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    # sequence 1 starts at block 2: position 140 lands in block 3 = out of range
-    mla.append_cache(cache, torch.tensor([0, 2], device=dev), torch.tensor([0, 1], dtype=torch.int32, device=dev),
-                     torch.tensor([3, 140], dtype=torch.int32, device=dev), c, k, tab, st)
+    # table rows of 2 blocks; sequence 1's second entry (block 7) is outside the 3-block pool, and
+    # position 300 of sequence 0 is past its row (300 // 128 = 2)
+    table = torch.tensor([[0, 1], [2, 7]], dtype=torch.int32, device=dev)
+    mla.append_cache(cache, table, torch.tensor([0, 1, 0], dtype=torch.int32, device=dev),
+                     torch.tensor([3, 140, 255], dtype=torch.int32, device=dev), c, k, tab, st)
     torch.cuda.synchronize()
-    assert int(st.item()) & 0x1
+    assert int(st.item()) == 0x1
+    # a sequence index outside the table's rows is reported, and its row is never read
+    mla.append_cache(cache, table, torch.tensor([2, -1], dtype=torch.int32, device=dev),
+                     torch.tensor([0, 0], dtype=torch.int32, device=dev), c[:2], k[:2], tab, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0x1
     u = H.cache_u16(cache)
     assert np.any(H.unpack_rows(u, [0], [3]) != 0)
     assert np.all(u[1:] == 0)
     st.zero_()
-    mla.append_cache(cache, torch.tensor([0], device=dev), torch.tensor([0], dtype=torch.int32, device=dev),
+    mla.append_cache(cache, table, torch.tensor([0], dtype=torch.int32, device=dev),
                      torch.tensor([9], dtype=torch.int32, device=dev), c[:1], k[:1], tab[:5], st)
     torch.cuda.synchronize()
     assert int(st.item()) & 0x2
@@ -280,6 +291,64 @@ def test_decode_reports_short_kv_len(cuda_ok, H):
     prob.decode(prob.absorb())
     torch.cuda.synchronize()
     assert int(prob.status.item()) & 0x4
+
+
+# ----------------------------------------------------------------- paged cache
+
+def test_decode_paged_shuffled_tables_match_contiguous_and_oracle(cuda_ok, H):
+    """Sequences whose blocks are scattered over the pool in random order, with table entries past each
+    sequence's blocks naming NaN-filled unowned blocks: the same results, bit for bit, as the contiguous
+    layout (the kernels compute tile by tile, wherever the tile lives) and within the bar of the oracle."""
+    cfg = mi.MLAConfig("paged", B=9, H=128, n_q=2, L=None, L_max=1300, seed=4242)
+    flat = H.build_problem(cfg)
+    paged = H.build_problem(cfg, shuffle_seed=7, extra_cols=3)
+    assert not np.array_equal(paged.tables[:, 0], flat.tables[:, 0])
+    q = flat.absorb()
+    out_f, lse_f = flat.decode(q)
+    out_p, lse_p = paged.decode(q)
+    torch.cuda.synchronize()
+    assert int(flat.status.item()) == 0 and int(paged.status.item()) == 0
+    assert torch.equal(out_f, out_p) and torch.equal(lse_f, lse_p)
+    _check_decode(paged, out_p, lse_p, range(cfg.B), heads=range(0, 128, 11), label="paged")
+    out_c, _ = paged.decode(q, num_splits=2, path="cudacore")
+    torch.cuda.synchronize()
+    assert int(paged.status.item()) == 0
+    a, b = out_p.float().cpu().numpy(), out_c.float().cpu().numpy()
+    assert np.all(np.abs(a - b) <= 2e-3 + 2 ** -6 * np.abs(b))
+
+
+def test_decode_paged_v2_time_shape_sampled(cuda_ok, H):
+    """V2-shaped workload on a shuffled pool (512 blocks of 32 sequences in random order)."""
+    cfg = mi.CONFIGS["v2"]
+    prob = H.build_problem(cfg, shuffle_seed=11)
+    out, lse = prob.decode(prob.absorb())
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    _check_decode(prob, out, lse, [5, 30], heads=range(3, 128, 25), label="v2 paged")
+
+
+def test_decode_table_overflow_and_bad_entry_are_reported(cuda_ok, H):
+    """A sequence longer than its table row is not processed (zero rows, lse -inf, ROW_RANGE); the others
+    are unaffected.  A table entry outside the pool is reported and never dereferenced."""
+    import mla_latent_kv_34_b200 as mla
+    cfg = mi.MLAConfig("overflow", B=3, H=16, n_q=1, L=None, L_max=600, seed=8)
+    prob = H.build_problem(cfg, lengths=[300, 200, 130])
+    q = prob.absorb()
+    kv = prob.kv_len.clone()
+    kv[1] = 3 * 128 + 1  # needs 4 blocks; the rows hold 3
+    lse = torch.empty((cfg.T, cfg.H), dtype=torch.float32, device="cuda")
+    out = mla.decode(q, prob.cache, prob.block_table, kv, prob.W_UV, cfg.n_q, cfg.scale, lse_out=lse,
+                     dev_status=prob.status)
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0x1
+    assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+    _check_decode(prob, out, lse, [0, 2], label="overflow")
+    prob.status.zero_()
+    bad = prob.block_table.clone()
+    bad[2, 1] = prob.cache.shape[0] + 5
+    mla.decode(q, prob.cache, bad, prob.kv_len, prob.W_UV, cfg.n_q, cfg.scale, lse_out=lse, dev_status=prob.status)
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0x1
 
 
 # ----------------------------------------------------------------- combine
