@@ -118,7 +118,7 @@ def test_append_out_of_range_is_reported_and_skipped(cuda_ok, H):
     # position 300 of sequence 0 is past its row (300 // 128 = 2)
     table = torch.tensor([[0, 1], [2, 7]], dtype=torch.int32, device=dev)
     mla.append_cache(cache, table, torch.tensor([0, 1, 0], dtype=torch.int32, device=dev),
-                     torch.tensor([3, 140, 255], dtype=torch.int32, device=dev), c, k, tab, st)
+                     torch.tensor([3, 140, 300], dtype=torch.int32, device=dev), c, k, tab, st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0x1
     # a sequence index outside the table's rows is reported, and its row is never read
