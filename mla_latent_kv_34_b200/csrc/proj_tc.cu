@@ -261,7 +261,14 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
         p_last = static_cast<int>((static_cast<int64_t>(ts + ntb) * P_g - 1) / Nt);
     }
     const int64_t seg0 = static_cast<int64_t>(g) * slots + b;  // slot of piece p: seg0 + p
+    // with more pairs than tiles some pairs in [p_first, p_last] have empty ranges and wrote nothing
+    auto live = [&](int p) {
+        const int lo = static_cast<int>((static_cast<int64_t>(p) * Nt) / P_g);
+        const int hi = static_cast<int>((static_cast<int64_t>(p + 1) * Nt) / P_g);
+        return max(lo, ts) < min(hi, ts + ntb);
+    };
     for (int p = p_first; p <= p_last; ++p) {
+        if (!live(p)) continue;
         const float2 ml = ml_part[(seg0 + p) * 128 + r];
         if (ml.x == -CUDART_INF_F) continue;
         const float Mn = fmaxf(M, ml.x);
@@ -273,6 +280,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     for (int i = 0; i < 32; ++i) acc[i] = 0.f;
     const int cg0 = 32 * qtr + 8 * k;
     for (int p = p_first; p <= p_last; ++p) {
+        if (!live(p)) continue;
         const float mp = ml_part[(seg0 + p) * 128 + r].x;
         if (mp == -CUDART_INF_F) continue;
         const float w = exp2f(mp - M);
