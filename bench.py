@@ -69,6 +69,10 @@ def parse_args(argv=None):
                     help="skip the separate timing of the compressed-query up-projection")
     ap.add_argument("--query-rank", type=int, default=1536, help="d_c' of the query up-projection timing")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle samples")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the separate timing of prefill chunks (naive vs absorbed form)")
+    ap.add_argument("--prefill-config", default="v2",
+                    help="workload whose first sequence the prefill chunks are timed on (N=1 only)")
     return ap.parse_args(argv)
 
 
@@ -443,6 +447,79 @@ def measure_query_up(torch, mla, cfg, dev, time_graph, n, peaks, d_cq):
             "note": "timed alone, L2 flushed before each launch; not part of the step"}
 
 
+def prefill_flops(L: int, n: int, H: int) -> dict:
+    """Algorithmic FLOPs of the last n of L tokens of one sequence attending causally, in both forms.
+
+    naive: rebuild k^C and v^C of every key and head (2 x 128 x 512 MACs), then 192 + 128 MACs per
+    (query, visible key, head).  absorbed: W^UK into each query and W^UV after (2 x 128 x 512 MACs per
+    (query, head)), then 576 + 512 MACs per (query, visible key, head).
+    """
+    visible = n * (L - n) + n * (n + 1) // 2
+    return {"naive": 2 * (L * H * 2 * 128 * 512 + visible * H * (192 + 128)),
+            "absorbed": 2 * (n * H * 2 * 128 * 512 + visible * H * (576 + 512))}
+
+
+def measure_prefill(torch, mla, cfg, st, dev, time_graph, steps, peaks, chunks=(64, 128, 256, 512, 1024)):
+    """Time one prefill chunk of n new tokens at the end of sequence 0 in both forms: mla_prefill_naive
+    (decompress + attend) and, for n <= 256, the absorbed path (absorb_q + decode with n_q = n).  Each is a
+    CUDA graph timed alone with L2 flushed before each launch; not part of the step."""
+    L = int(st["lengths"][0])
+    H = cfg.H
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    row = st["block_table"][0].contiguous()
+    table1 = row.reshape(1, -1)
+    kv1 = torch.full((1,), L, dtype=torch.int32, device=dev)
+    res = {"L": L, "H": H, "launches": steps, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "chunks": []}
+
+    def dbf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    def timed(run):
+        for _ in range(3):
+            run()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            run()
+        torch.cuda.synchronize()
+        us = 1e3 * statistics.mean(time_graph(g, steps))
+        del g
+        return us
+
+    ws_naive = torch.empty(mla.prefill_workspace_bytes(L, H), dtype=torch.uint8, device=dev)
+    for n in chunks:
+        if n > L:
+            continue
+        qcfg = mi.MLAConfig("prefill", B=1, H=H, n_q=n, L=L, seed=cfg.seed + 991)
+        qn_bits, qr_bits = mi.queries(qcfg)
+        qn, qr = dbf(qn_bits), dbf(qr_bits)
+        out = torch.empty((n, H, mi.D_H), dtype=torch.bfloat16, device=dev)
+        f = prefill_flops(L, n, H)
+        ent = {"n": n}
+        us = timed(lambda: mla.prefill_naive(qn, qr, st["rope"], st["cache"], row, L, st["W_UK"], st["W_UV"],
+                                             cfg.scale, workspace=ws_naive, out=out, dev_status=status))
+        ent["naive_us"] = round(us, 2)
+        ent["naive_tflops"] = round(f["naive"] / (us * 1e-6) / 1e12, 1)
+        if n <= 256:
+            pos = torch.arange(L - n, L, dtype=torch.int32, device=dev)
+            qa = torch.empty((n, H, mi.D_ROW), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(mla.decode_workspace_bytes(1, n, H), dtype=torch.uint8, device=dev)
+
+            def absorbed():
+                mla.absorb_q(qn, qr, pos, st["W_UK"], st["rope"], q_out=qa, dev_status=status)
+                mla.decode(qa, st["cache"], table1, kv1, st["W_UV"], n, cfg.scale, workspace=ws, out=out,
+                           dev_status=status)
+            us = timed(absorbed)
+            ent["absorbed_us"] = round(us, 2)
+            ent["absorbed_tflops"] = round(f["absorbed"] / (us * 1e-6) / 1e12, 1)
+            ent["faster"] = "naive" if ent["naive_us"] < ent["absorbed_us"] else "absorbed"
+        res["chunks"].append(ent)
+    if int(status.item()) != 0:
+        return {"error": "device status " + mla.device_status_string(int(status.item()))}
+    res["note"] = ("naive: decompress k^C, v^C of all L keys then causal attention; absorbed: absorb_q + the "
+                   "decode kernels with n_q = n (n <= 256); timed alone, L2 flushed before each launch")
+    return res
+
+
 def _check_status(mla, st):
     if int(st["status"].item()) != 0:
         raise SystemExit(f"device status {mla.device_status_string(int(st['status'].item()))}")
@@ -534,6 +611,11 @@ def measure_workload(torch, mla, dist, cfg, dev, args, flush, sampler=None, head
         "step_roofline_frac": round(step_roof_s / (ms_per_step * 1e-3), 4),
         "roofline": roofline, "e2e": e2e,
     }
+    if dist.world == 1 and not args.no_prefill and cfg.name == args.prefill_config:
+        try:
+            res["prefill"] = measure_prefill(torch, mla, cfg, st, dev, time_graph, min(args.steps, 50), peaks)
+        except Exception as e:  # reported in the line; the step's numbers stand on their own
+            res["prefill"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     if headline and dist.world == 1 and not args.no_query_up:
         try:
             res["query_up"] = measure_query_up(torch, mla, cfg, dev, time_graph, min(args.steps, 1000), peaks,
@@ -569,12 +651,15 @@ def run_ours(args, dist):
         clocks["window"] = (f"the timed steps plus untimed replays of the same step graph, "
                             f"{head['loaded_s']:.2f} s of load in all")
     per_config = {}
+    prefill = head.get("prefill")
     extras = [c for c in args.extra_configs.split(",") if c and c != args.config] if dist.world == 1 else []
     for name in extras:
         r = measure_workload(torch, mla, dist, rank_config(mi.CONFIGS[name], dist.rank), dev, args, flush)
         per_config[name] = {k: r[k] for k in ("workload", "us_per_step", "kernel_us", "tflops",
                                               "cache_tokens_per_s", "step_roofline_frac", "roofline", "e2e")}
         per_config[name]["value"] = round(r["value"], 4)
+        if "prefill" in r:
+            prefill = r["prefill"]
         per_config[name]["unit"] = UNIT
 
     counts = head["counts"]
@@ -599,6 +684,8 @@ def run_ours(args, dist):
         line["per_config"] = per_config
     if "query_up" in head:
         line["query_up"] = head["query_up"]
+    if prefill is not None:
+        line["prefill"] = prefill
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, head["lengths"], args.cpu_seconds)
     dist.close()

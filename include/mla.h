@@ -20,11 +20,13 @@
  * queries are compressed), mla_absorb_q, mla_append_cache, mla_decode (=
  * mla_decode_attend + mla_decode_finish; mla_decode_static without a
  * workspace), with mla_decode_cudacore + mla_splitkv_combine as an
- * independent CUDA-core path of the same decode.
+ * independent CUDA-core path of the same decode.  Long prefill chunks use
+ * mla_prefill_naive (the naive form) after mla_append_cache.
  *
  * Fixed sizes: d_c = 512, d_h^R = 64, d_h = 128 (cached row D = 576).
  * Runtime sizes: B sequences, H heads (1..128), n_q new query tokens per
- * sequence (1..16), T = B * n_q query rows (row t = b * n_q + j).
+ * sequence (1..256: a decode step, speculative tokens or a prefill chunk),
+ * T = B * n_q query rows (row t = b * n_q + j).
  *
  * Latent cache layout (paged, blocked).  The cache is a pool of blocks of
  * MLA_BLOCK_TOKENS = 128 tokens, MLA_BLOCK_BYTES = 147456 bytes each, and a
@@ -185,8 +187,9 @@ mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int32_t* bloc
  * mla_decode_workspace_bytes -- device workspace mla_decode needs for these
  * sizes (num_splits as passed to mla_decode; 0 = automatic).  It holds the
  * attend phase's pieces (a slot of 128 rows x (512 fp32 + max, sum) per
- * sequence plus one per CTA pair, at most 74 pairs, per group of 128 query
- * rows) and the merged latent output in bf16 ([H, ~B*n_q, 512]).
+ * sequence plus one per CTA pair of the group, for each group of 128 query
+ * rows; with G groups a group gets at most max(1, 74 / G) pairs) and the
+ * merged latent output in bf16 ([H, ~B*n_q, 512]).
  */
 size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
 
@@ -298,6 +301,45 @@ mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_blo
                                int B, int n_q, int H, float scale, int num_splits,
                                void* workspace, size_t ws_bytes, void* out, float* lse_out,
                                int32_t* dev_status, mla_stream stream);
+
+/*
+ * mla_prefill_workspace_bytes / mla_prefill_naive -- attention of n new tokens
+ * of one sequence in the NAIVE form, for long prefill chunks.  ("两张账" page,
+ * "第一张账": the naive path rebuilds k^C = W^UK c and v^C = W^UV c from c^KV;
+ * MLA explainer 2.2.2: attention on [q^C; R q^R].[k^C; k^R].)  The absorbed
+ * form of mla_decode does 3.4x the arithmetic per (query, key, head), so for
+ * causal chunks beyond ~340 tokens rebuilding the keys and values once per
+ * (key, head) costs less.
+ *   q_nope, q_rope  bf16 [n, H, 128] / [n, H, 64]: the chunk's queries, q^R
+ *                   unrotated (rotated here at its position, as mla_absorb_q)
+ *   rope_table      fp32 [rope_len, 64] (as for mla_append_cache); rope_len >= L
+ *   cache           pool of cap_blocks blocks (layout above) holding the
+ *                   sequence's L tokens, the n new ones (already appended) last
+ *   blocks          int32 [ceil(L / 128)], device: the sequence's row of the
+ *                   block table (tile i = pool block blocks[i])
+ *   query j sits at position L - n + j and sees keys 0 .. L - n + j
+ *   W_UK, W_UV      bf16 [H, 128, 512]
+ *   workspace       mla_prefill_workspace_bytes(L, H) bytes: the rebuilt
+ *                   k^C and v^C of every key and head, bf16 [L, H, 128] each
+ *   out             bf16 [n, H, 128];  lse_out fp32 [n, H] or NULL
+ * Two kernels: the decompression (tcgen05, D[token, 0..255] = c . [W^UK_h ;
+ * W^UV_h]^T per 128-token block and head), then causal attention (tcgen05 QK^T
+ * and PV, online softmax in fp32, one CTA per head and 128-query tile).
+ * Rounding: k^C, v^C, the rotated q^R and P are bf16; sums and softmax fp32.
+ * Errors (before any launch): MLA_ERR_INVALID_ARG for n > L, L > rope_len, a
+ * bad scale, cap_blocks < 1, null or misaligned pointers;
+ * MLA_ERR_UNSUPPORTED_SHAPE for H outside 1..128 or L * H * 128 >= 2^31;
+ * MLA_ERR_WORKSPACE.  A block entry outside [0, cap_blocks) sets
+ * MLA_DEVERR_ROW_RANGE (results unspecified); an expired bounded wait sets
+ * MLA_DEVERR_TIMEOUT.  n = 0 launches nothing.
+ */
+size_t mla_prefill_workspace_bytes(int L, int H);
+mla_status mla_prefill_naive(const void* q_nope, const void* q_rope, const float* rope_table,
+                             int64_t rope_len, const void* cache, int64_t cap_blocks,
+                             const int32_t* blocks, int L, int n, const void* W_UK,
+                             const void* W_UV, int H, float scale, void* workspace,
+                             size_t ws_bytes, void* out, float* lse_out, int32_t* dev_status,
+                             mla_stream stream);
 
 /*
  * mla_splitkv_combine -- log-sum-exp merge of split-KV partials.

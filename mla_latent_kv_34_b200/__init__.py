@@ -45,6 +45,9 @@ _SIGS = {
     "mla_decode_cudacore": ([_p, _p, _i64, _p, _i32, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p,
                              _p], _i32),
     "mla_splitkv_combine": ([_p, _p, _i32, _i32, _i32, _p, _p, _p, _p], _i32),
+    "mla_prefill_workspace_bytes": ([_i32, _i32], _sz),
+    "mla_prefill_naive": ([_p, _p, _p, _i64, _p, _i64, _p, _i32, _i32, _p, _p, _i32, _f32, _p, _sz, _p, _p, _p, _p],
+                          _i32),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -281,4 +284,33 @@ def splitkv_combine(o_part, lse_part, W_UV=None, out=None, lse_out=None, stream=
         _ptr(o_part, torch.float32, (T, H, S, D_C), "o_part"), _ptr(lse_part, torch.float32, (T, H, S), "lse_part"),
         T, H, S, _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), _ptr(out, None, None, "out"),
         _ptr(lse_out, torch.float32, (T, H), "lse_out"), _stream(stream)))
+    return out
+
+
+def prefill_workspace_bytes(L: int, H: int) -> int:
+    return int(lib.mla_prefill_workspace_bytes(L, H))
+
+
+def prefill_naive(q_nope, q_rope, rope_tab, cache, blocks, L: int, W_UK, W_UV, scale: float,
+                  workspace=None, out=None, lse_out=None, dev_status=None, stream=None):
+    """Naive-form attention of the last n = len(q_nope) of a sequence's L cached tokens -> bf16 [n, H, 128].
+
+    ``blocks``: int32 device tensor, the sequence's row of the block table (at least ceil(L / 128) entries).
+    """
+    n, H = q_nope.shape[0], q_nope.shape[1]
+    if blocks.dim() != 1 or blocks.shape[0] * BLOCK_TOKENS < L:
+        raise MLAError("blocks must be an int32 vector of at least ceil(L / 128) entries")
+    need = prefill_workspace_bytes(L, H)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
+    if out is None:
+        out = torch.empty((n, H, D_H), dtype=torch.bfloat16, device=q_nope.device)
+    _check(lib.mla_prefill_naive(
+        _ptr(q_nope, torch.bfloat16, (n, H, D_H), "q_nope"), _ptr(q_rope, torch.bfloat16, (n, H, D_R), "q_rope"),
+        _ptr(rope_tab, torch.float32, None, "rope_table"), rope_tab.shape[0], _cache_ptr(cache), cache.shape[0],
+        _ptr(blocks, torch.int32, None, "blocks"), int(L), n, _ptr(W_UK, torch.bfloat16, (H, D_H, D_C), "W_UK"),
+        _ptr(W_UV, torch.bfloat16, (H, D_H, D_C), "W_UV"), H, float(scale), _ptr(workspace, None, None, "workspace"),
+        workspace.numel() * workspace.element_size(), _ptr(out, torch.bfloat16, (n, H, D_H), "out"),
+        _ptr(lse_out, torch.float32, (n, H), "lse_out"), _ptr(dev_status, torch.int32, None, "dev_status"),
+        _stream(stream)))
     return out

@@ -34,10 +34,12 @@ DecodeWs decode_ws_layout(int B, int n_q, int H, int S) {
 
 mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
+int max_pairs_per_group(int G) { return kMaxPairs / G > 1 ? kMaxPairs / G : 1; }
+
 // ---- tensor-core path: segment partials [G][slots][128 rows] float2 (m, l), then (1024-aligned)
 //      [G][slots] blocks of 128 rows x 512 fp32 O, each stored as [128 column groups of 4][128 rows] x float4,
 //      then (1024-aligned) the merged latent output o_lat as bf16 operand tiles, [H][olat_rows(T)] x 1 KB.
-//      A slot per (sequence + CTA pair): a pair's tile range starts at most one piece into a sequence.
+//      A slot per (sequence + CTA pair of the group): a pair's range starts at most one piece into a sequence.
 struct TcWs {
     int G, slots;
     size_t ml_part, o_part, olat, total;
@@ -48,7 +50,8 @@ size_t align1k(size_t x) { return ((x + 1023) / 1024) * 1024; }
 TcWs tc_ws_layout(int B, int n_q, int H) {
     TcWs w;
     w.G = (n_q * H + 127) / 128;
-    w.slots = B + kMaxPairs;
+    // a group gets at most max(1, kMaxPairs / G) CTA pairs (long query chunks: many groups, few pairs each)
+    w.slots = B + max_pairs_per_group(w.G);
     const size_t rows = static_cast<size_t>(w.G) * w.slots * 128;
     w.ml_part = 0;
     w.o_part = align1k(rows * sizeof(float2));
@@ -63,7 +66,7 @@ int tc_clusters_per_group(int G, int num_splits) {
     int pg = total / G;
     if (pg < 1) pg = 1;
     if (num_splits > 0 && num_splits < pg) pg = num_splits;
-    return pg;
+    return pg < max_pairs_per_group(G) ? pg : max_pairs_per_group(G);
 }
 
 constexpr int64_t kMaxPoolBlocks = 0x7FFFFFFF;                 // block-table entries are int32
@@ -257,6 +260,37 @@ mla_status mla_decode_cudacore(const void* q, const void* cache, int64_t cap_blo
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     return cuda_status(launch_combine(o_part, lse_part, B * n_q, H, S, static_cast<const uint16_t*>(W_UV), out,
                                       lse_out, cs));
+}
+
+size_t mla_prefill_workspace_bytes(int L, int H) {
+    if (L < 1 || H < 1) return 0;
+    return 2 * prefill_rows_bytes(L, H);
+}
+
+mla_status mla_prefill_naive(const void* q_nope, const void* q_rope, const float* rope_table, int64_t rope_len,
+                             const void* cache, int64_t cap_blocks, const int32_t* blocks, int L, int n,
+                             const void* W_UK, const void* W_UV, int H, float scale, void* workspace,
+                             size_t ws_bytes, void* out, float* lse_out, int32_t* dev_status, mla_stream stream) {
+    if (n < 0 || L < 0 || cap_blocks < 0 || cap_blocks > kMaxPoolBlocks || rope_len < 0) return MLA_ERR_INVALID_ARG;
+    if (H < 1 || H > kMaxHeads) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (n == 0) return MLA_OK;
+    if (n > L || L > rope_len || L >= (1 << 30) || cap_blocks < 1) return MLA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(L) * H * kDh >= (int64_t(1) << 31)) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (!(scale > 0.f) || !isfinite(scale)) return MLA_ERR_INVALID_ARG;
+    if (!q_nope || !q_rope || !rope_table || !cache || !blocks || !W_UK || !W_UV || !workspace || !out)
+        return MLA_ERR_INVALID_ARG;
+    if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(rope_table) || !aligned16(cache) ||
+        !aligned16(W_UK) || !aligned16(W_UV) || !aligned16(workspace) || !aligned16(out))
+        return MLA_ERR_INVALID_ARG;
+    const size_t rows = prefill_rows_bytes(L, H);
+    if (ws_bytes < 2 * rows) return MLA_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    return cuda_status(launch_prefill_naive(
+        static_cast<const uint16_t*>(q_nope), static_cast<const uint16_t*>(q_rope), rope_table,
+        static_cast<const uint8_t*>(cache), cap_blocks, blocks, L, n, static_cast<const uint16_t*>(W_UK),
+        static_cast<const uint16_t*>(W_UV), H, scale, reinterpret_cast<uint16_t*>(ws),
+        reinterpret_cast<uint16_t*>(ws + rows), static_cast<uint16_t*>(out), lse_out, dev_status,
+        static_cast<cudaStream_t>(stream)));
 }
 
 mla_status mla_splitkv_combine(const float* o_part, const float* lse_part, int T, int H, int num_splits,

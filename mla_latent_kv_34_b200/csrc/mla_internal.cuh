@@ -14,7 +14,7 @@ constexpr int kDr = 64;            // RoPE width d_h^R
 constexpr int kDh = 128;           // head width d_h
 constexpr int kRow = kDc + kDr;    // packed cache row (576 bf16 = 1152 B)
 constexpr int kMaxHeads = 128;
-constexpr int kMaxNq = 16;
+constexpr int kMaxNq = 256;       // new query tokens per sequence (decode, speculation, prefill chunks)
 constexpr int kBlockTokens = MLA_BLOCK_TOKENS;  // tokens per cache block
 constexpr int kBlockBytes = MLA_BLOCK_BYTES;    // 9 chunks x [128 rows x 128 B]
 constexpr int kBlockChunk = kBlockTokens * 128;  // bytes of one 64-column chunk of a block
@@ -69,6 +69,14 @@ cudaError_t launch_absorb_tc(const uint16_t* q_nope, const uint16_t* q_rope, con
 // Query up-projections q^C = W^UQ c^Q, q^R = W^QR c^Q (query_up.cu).
 cudaError_t launch_query_up(const uint16_t* c_q, const uint16_t* W_UQ, const uint16_t* W_QR, int T, int H, int d_cq,
                             uint16_t* q_nope, uint16_t* q_rope, int32_t* dev_status, cudaStream_t stream);
+
+// Naive-form attention for long prefill chunks (prefill_naive.cu).
+size_t prefill_rows_bytes(int L, int H);
+cudaError_t launch_prefill_naive(const uint16_t* q_nope, const uint16_t* q_rope, const float* rope_table,
+                                 const uint8_t* cache, int64_t cap_blocks, const int32_t* blocks, int L, int n,
+                                 const uint16_t* W_UK, const uint16_t* W_UV, int H, float scale, uint16_t* k_rows,
+                                 uint16_t* v_rows, uint16_t* out, float* lse_out, int32_t* dev_status,
+                                 cudaStream_t stream);
 
 cudaError_t launch_decode_simt(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
                                int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale, int splits,

@@ -205,6 +205,22 @@ def test_decode_multi_token_queries(cuda_ok, H, n_q, Hh, L):
     _check_decode(prob, out, lse, [0, 1, 2], label=f"n_q={n_q}")
 
 
+@pytest.mark.parametrize("n_q,Hh,L", [(32, 16, 600), (100, 8, 400), (256, 16, 700), (64, 128, 300)])
+def test_decode_prefill_chunks(cuda_ok, H, n_q, Hh, L):
+    """Chunks of up to 256 new tokens per sequence in the absorbed form (the arithmetic favours it
+    over the naive form below about 340 tokens); query j sees keys up to L - n_q + j."""
+    cfg = mi.MLAConfig("chunk", B=2, H=Hh, n_q=n_q, L=L, seed=3000 + n_q + Hh)
+    prob = H.build_problem(cfg, lengths=[L, max(n_q, L // 2)], shuffle_seed=n_q)
+    q = prob.absorb()
+    out, lse = prob.decode(q)
+    ref_out, _ = prob.decode(q, num_splits=2, path="cudacore")
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    a, b = out.float().cpu().numpy(), ref_out.float().cpu().numpy()
+    assert np.all(np.abs(a - b) <= 2 * (ATOL + RTOL * np.abs(b)))
+    _check_decode(prob, out, lse, [0, 1], heads=range(0, Hh, max(1, Hh // 8)), label=f"chunk n_q={n_q}")
+
+
 def test_decode_small_ragged_full(cuda_ok, H):
     cfg = mi.MLAConfig("ragged-small", B=12, H=128, n_q=2, L=None, L_max=700, seed=77)
     prob = H.build_problem(cfg)
