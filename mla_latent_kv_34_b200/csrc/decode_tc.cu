@@ -67,14 +67,15 @@ constexpr int kVPerTile = 8 / kVChunksPerStage;  // V stages per tile (the 8 lat
 constexpr int kVStages = 2;          // O CTA: ring of V stages
 constexpr int kPBytes = kRows * kTile * 2;       // 32 KB bf16 P tile: two [128 x 64] swizzled atoms
 constexpr int kMsgBytes = kPBytes + kRows * 4;  // P | alpha[128] (per-row rescale factors): one bulk copy
-constexpr int kMsgStride = 33792;    // 1024-aligned message slots in the O CTA
+constexpr int kMsgStride = 33792;    // 1024-aligned message slots (P atoms must start 1024-aligned)
+constexpr int kPSlots = 3;           // O CTA: message slots, so P(t) can land while P V(t-2) still runs
 constexpr int kSoftWarps = 8;        // S CTA: two warps per TMEM lane quadrant
 constexpr int kSoftThreads = kSoftWarps * 32;
 constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpSender = 10;
 constexpr int kThreads = 352;
 constexpr int kSyncThreads = kSoftThreads + 32;  // softmax warps + the sender warp
 // named barriers, S CTA: 1..4 the two warps of a TMEM lane quadrant; the rest over kSyncThreads
-constexpr uint32_t kNbFail = 6, kNbStaged = 7, kNbStageFree = 8;
+constexpr uint32_t kNbQFree = 5, kNbFail = 6, kNbStaged = 7, kNbStageFree = 8;
 constexpr uint64_t kLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleLog2 = 8.0f;
 static_assert(kKvChunks % kCopyChunks == 0, "a tile is a whole number of copies");
@@ -85,30 +86,36 @@ constexpr uint32_t kColQ = 0;     // S CTA: latent Q rows, 256 columns of packed
 constexpr uint32_t kColS0 = 256;  // S CTA: two 128-column score buffers (256, 384)
 __device__ __forceinline__ uint32_t col_s(uint32_t sb) { return kColS0 + 128u * sb; }
 
-// shared memory, S CTA
-constexpr int kSOffRing = 0;                                  // 4 x 48 KB
+// shared memory, S CTA.  P messages are built in two staging buffers, so the softmax can stage P(t+1)
+// while the copy of P(t) is still queued behind tile loads on this SM's copy engine; staging buffer 1
+// shares its space with the Q transpose tiles, used only while a segment's queries are reloaded.
+constexpr int kSOffRing = 0;                                  // 3 x 48 KB
 constexpr int kSOffQR = kRingSlots * kCopyBytes;              // RoPE part of Q: [128 x 64] swizzled, 16 KB
-constexpr int kSOffStage = kSOffQR + kRows * 128;             // the P message being built (kMsgBytes)
-constexpr int kSOffXchg = kSOffStage + kMsgStride;            // [2][128] fp32 half-row maxima / sums
+constexpr int kSOffStage0 = kSOffQR + kRows * 128;            // P message staging buffer 0 (kMsgBytes)
+constexpr int kSOffXchg = kSOffStage0 + kMsgStride;           // [2][128] fp32 half-row maxima / sums
 constexpr int kSOffQT = kSOffXchg + 2 * kRows * 4;            // 8 warps x [32 rows x 128 B] Q transpose tiles
-constexpr int kSOffBar = kSOffQT + kSoftWarps * 32 * 128;
+constexpr int kSOffStage1 = kSOffQT;                          //   = P message staging buffer 1
+constexpr int kQTBytes = kSoftWarps * 32 * 128;
+constexpr int kSOffBar = kSOffQT + (kQTBytes > kMsgBytes ? kQTBytes : kMsgBytes);
 constexpr int kSBarFull = 0, kSBarEmpty = kRingSlots, kSBarSFull = 2 * kRingSlots, kSBarSEmpty = kSBarSFull + 2,
-              kSBarPEmpty = kSBarSEmpty + 2, kSBarQReady = kSBarPEmpty + 2, kSBarFin = kSBarQReady + 1,
+              kSBarPEmpty = kSBarSEmpty + 2, kSBarQReady = kSBarPEmpty + kPSlots, kSBarFin = kSBarQReady + 1,
               kSNumBars = kSBarFin + 1;
 constexpr int kSOffTail = kSOffBar + kSNumBars * 8;
-// shared memory, O CTA
+// shared memory, O CTA: the last message slot ends at its alpha values (no padding), barriers follow
 constexpr int kOOffV = 0;                                     // 2 x 64 KB
-constexpr int kOOffMsg = kVStages * kVStageBytes;             // 2 message slots
-constexpr int kOOffBar = kOOffMsg + 2 * kMsgStride;
-constexpr int kOBarVFull = 0, kOBarVEmpty = kVStages, kOBarPFull = 2 * kVStages, kOBarOFull = kOBarPFull + 2,
+constexpr int kOOffMsg = kVStages * kVStageBytes;             // kPSlots message slots, kMsgStride apart
+constexpr int kOOffBar = kOOffMsg + (kPSlots - 1) * kMsgStride + kMsgBytes;
+constexpr int kOBarVFull = 0, kOBarVEmpty = kVStages, kOBarPFull = 2 * kVStages, kOBarOFull = kOBarPFull + kPSlots,
               kOBarOFree = kOBarOFull + 1, kOBarRescReq = kOBarOFree + 1, kOBarRescDone = kOBarRescReq + 1,
               kOBarODrain = kOBarRescDone + 1, kOBarFin = kOBarODrain + 1, kONumBars = kOBarFin + 1;
 constexpr int kOOffTail = kOOffBar + kONumBars * 8;
 constexpr int kTailBytes = 32;  // tmem base, abort flag, resc slot, tile total, first sequence and its tile
 constexpr int kSmemBytes = (kSOffTail > kOOffTail ? kSOffTail : kOOffTail) + kTailBytes;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kSOffQR % 1024 == 0 && kSOffStage % 1024 == 0 && kOOffMsg % 1024 == 0 && kMsgStride % 1024 == 0,
+static_assert(kSOffQR % 1024 == 0 && kSOffStage0 % 1024 == 0 && kSOffStage1 % 1024 == 0 && kOOffMsg % 1024 == 0 &&
+                  kMsgStride % 1024 == 0,
               "swizzle atoms 1024-aligned");
+static_assert(kOOffBar % 8 == 0 && kSOffBar % 8 == 0, "mbarriers 8-byte aligned");
 static_assert(kMsgBytes % 16 == 0, "bulk copy size");
 static_assert(kMsgStride >= kMsgBytes, "message slot");
 
@@ -224,8 +231,8 @@ decode_tc_kernel(const Params p) {
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&bars[kSBarSFull + i], 1);
                 mbar_init(&bars[kSBarSEmpty + i], kSoftThreads);
-                mbar_init(&bars[kSBarPEmpty + i], 1);
             }
+            for (int i = 0; i < kPSlots; ++i) mbar_init(&bars[kSBarPEmpty + i], 1);
             mbar_init(&bars[kSBarQReady], kSoftThreads);
             mbar_init(&bars[kSBarFin], 1);
         } else {
@@ -233,7 +240,7 @@ decode_tc_kernel(const Params p) {
                 mbar_init(&bars[kOBarVFull + i], 1);
                 mbar_init(&bars[kOBarVEmpty + i], 1);
             }
-            for (int i = 0; i < 2; ++i) mbar_init(&bars[kOBarPFull + i], 1);
+            for (int i = 0; i < kPSlots; ++i) mbar_init(&bars[kOBarPFull + i], 1);
             mbar_init(&bars[kOBarOFull], 1);
             mbar_init(&bars[kOBarOFree], kRows);
             mbar_init(&bars[kOBarRescReq], 1);
@@ -397,9 +404,6 @@ decode_tc_kernel(const Params p) {
             const int r = 32 * qd + lane;
             const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * qd) << 16);
             float* xchg = reinterpret_cast<float*>(smem + kSOffXchg);  // [2][128]
-            // this thread's row of P in the staged message: atom hf, row r (8 swizzled units)
-            uint8_t* stage = smem + kSOffStage;
-            uint8_t* prow = stage + hf * (kRows * 128) + r * 128;
             const int rr = g * kRows + r;
             const bool row_ok = rr < p.R;
             const int j = row_ok ? rr / p.H : 0;
@@ -424,7 +428,6 @@ decode_tc_kernel(const Params p) {
                 const char* nq = (have_next && row_ok) ? reinterpret_cast<const char*>(
                                                               p.q + (static_cast<int64_t>(sn.b) * p.R + rr) * kRow)
                                                         : nullptr;
-                __syncwarp();
                 {
                     uint8_t* qt = smem + kSOffQT + warp * (32 * 128);
                     const int lu = lane & 7, lr = lane >> 3;  // unit and row-in-quad of this lane's loads
@@ -440,6 +443,9 @@ decode_tc_kernel(const Params p) {
                                 if (g * kRows + 32 * qd + ri < p.R)
                                     x[j][i] = reinterpret_cast<const uint4*>(p.q + (qrow0 + ri) * kRow)[8 * (c + j) + lu];
                             }
+                        // the transpose tiles double as staging buffer 1: before the first write to them,
+                        // wait until the sender has seen every copy of earlier messages read out
+                        if (c == 4 * hf) bar_sync(kNbQFree, kSyncThreads);
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
 #pragma unroll
@@ -527,8 +533,10 @@ decode_tc_kernel(const Params p) {
                         failed = true;
                         break;
                     }
-                    // the sender has seen the previous tile's copy read the staging buffer
+                    // the sender has seen the copy that last used this staging buffer (tile n - 2) read it
                     bar_sync(kNbStageFree, kSyncThreads);
+                    uint8_t* stage = smem + ((n & 1u) ? kSOffStage1 : kSOffStage0);
+                    uint8_t* prow = stage + hf * (kRows * 128) + r * 128;
                     // P row r, columns 64hf.. -> atom hf, row r: 16-byte units u at (u ^ (r % 8))
 #pragma unroll
                     for (int u = 0; u < 8; ++u)
@@ -562,20 +570,27 @@ decode_tc_kernel(const Params p) {
             uint32_t n = 0;
             bool failed = false;
             while (!failed && w.next(p, s)) {
+                // every staged message read out before the Q reload reuses staging buffer 1
+                if (lane == 0) bulk_wait_group_read<0>();
+                __syncwarp();
+                bar_arrive(kNbQFree, kSyncThreads);
                 for (int t = s.t0; t < s.t1; ++t, ++n) {
-                    const uint32_t pb = n & 1u, up = n >> 1;
+                    const uint32_t pb = n % kPSlots, up = n / kPSlots;
                     if (bar_red_or(kNbFail, kSyncThreads, *abort_flag != 0)) {
                         failed = true;
                         break;
                     }
-                    if (lane == 0) bulk_wait_group_read<0>();
+                    // the copy of tile n - 2 (same staging buffer as tile n) has read its source; the copy of
+                    // tile n - 1 may still be queued
+                    if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
                     bar_arrive(kNbStageFree, kSyncThreads);
                     bar_sync(kNbStaged, kSyncThreads);
                     if (lane == 0) {
                         if (mbar_wait<true>(&bars[kSBarPEmpty + pb], (up & 1u) ^ 1u, abort_flag, kLimitNs)) {
                             mbar_arrive_expect_tx_remote(peer_pfull + 8 * pb, kMsgBytes);
-                            bulk_copy_to_peer(peer_msg + pb * kMsgStride, sbase + kSOffStage, kMsgBytes,
+                            bulk_copy_to_peer(peer_msg + pb * kMsgStride,
+                                              sbase + ((n & 1u) ? kSOffStage1 : kSOffStage0), kMsgBytes,
                                               peer_pfull + 8 * pb);
                             bulk_commit_group();
                         } else {
@@ -633,7 +648,7 @@ decode_tc_kernel(const Params p) {
             bool ok = true;
             while (ok && w.next(p, s)) {
                 for (int t = s.t0; ok && t < s.t1; ++t, ++n) {
-                    const uint32_t pb = n & 1u, up = n >> 1;
+                    const uint32_t pb = n % kPSlots, up = n / kPSlots;
                     const bool first = (t == s.t0);
                     if (lane == 0) {
                         ok = mbar_wait<true>(&bars[kOBarPFull + pb], up & 1u, abort_flag, kLimitNs);
