@@ -15,8 +15,8 @@
 // head and each moves a quarter of W^UK_h; the weight quarter lands as two TMA boxes
 // ([128 x 64] chunks, 128-byte swizzle) and is the MN-major A operand (M = latent
 // column, K = head dim) of 8 MMAs against the staged q_nope rows (N = rows).
-// merge: one CTA per (row group, sequence, quarter of the latent columns); a warp reads
-// 512 contiguous bytes of a piece at a time (the attend kernel's column-group order)
+// merge: one CTA per (32 latent columns, sequence, row group), four threads per row sharing the
+// sequence's pieces (the attend kernel writes them in [column group][row] order)
 // and writes o_lat into per-(head, 64-row block) tiles already in the swizzled K-major
 // operand layout, so the up-projection takes its operand with one bulk copy.
 // upproj: one CTA per (head, up to 64 rows); W^UV_h (eight [128 x 64] TMA boxes) is
@@ -202,7 +202,9 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
 
 // ------------------------------------------------------------------ merge
 
-constexpr int kMergeThreads = 512;  // 4 threads per row of the 128-row group, 8 column groups each
+constexpr int kMergeSplit = 4;                       // threads per row, each taking every 4th piece
+constexpr int kMergeThreads = 128 * kMergeSplit;     // a warp = 8 rows x 4 threads
+constexpr int kMergeSlices = 16;    // a CTA merges 32 of the 512 latent columns (8 column groups of 4)
 
 // Byte offset of row t of head h, latent unit (chunk c, unit u) in the o_lat tiles: per head, the rows
 // are cut into blocks of 64 (the last one olat_rows(T) - 64 * (blocks - 1) rows); a block is eight
@@ -214,14 +216,18 @@ __device__ __forceinline__ int64_t olat_offset(int T, int h, int t, int c, int u
     return (static_cast<int64_t>(h) * Tp + 64 * tb) * 1024 + c * rows * 128 + swz(i, u);
 }
 
+// One CTA per (32-column slice, sequence, row group).  Row r of the group is merged by four threads,
+// lanes 4 (r % 8) .. + 3 of warp r / 8, each over every fourth piece of the sequence with its own running
+// maximum; the four partial results are combined with warp shuffles.  A thread's loads of one piece are
+// eight 16-byte column groups of its row (the attend kernel's [column group][row] order).
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const float* __restrict__ o_part, const float2* __restrict__ ml_part, const int32_t* __restrict__ kv_len,
     int max_blocks, int B, int n_q, int H, int P_g, int slots, uint8_t* __restrict__ olat, float* __restrict__ lse_out) {
     __shared__ int red[2][kMergeThreads / 32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qtr = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
-    const int r = tid & 127, k = tid >> 7;  // row of the group; column groups 32 qtr + 8 k .. + 7
-    grid_dependency_wait();                 // the pieces come from the attend kernel
+    const int slice = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
+    const int r = 8 * warp + (lane >> 2), k = lane & 3;
+    grid_dependency_wait();  // the pieces come from the attend kernel
     grid_dependents_launch();
     // tiles of all sequences (the attend kernel's range split depends on the total) and before b
     int s_all = 0, s_pre = 0;
@@ -249,14 +255,10 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const int ntb = valid_seq_tiles(kv_len[b], n_q, max_blocks);
     const int R = n_q * H;
     const int rr = g * 128 + r;
-    if (rr >= R) return;
-    const int j = rr / H, h = rr % H;
-    const int t = b * n_q + j;
-    const int T = B * n_q;
+    const bool row_ok = rr < R;  // (no early exit: the shuffles below need every lane)
     // pieces of sequence b: the attend kernel's pairs whose tile range [lo, hi) meets [ts, ts + ntb)
-    float M = -CUDART_INF_F, z = 0.f;
     int p_first = 0, p_last = -1;
-    if (ntb > 0 && Nt > 0) {
+    if (ntb > 0 && Nt > 0 && row_ok) {
         p_first = static_cast<int>((static_cast<int64_t>(ts + 1) * P_g - 1) / Nt);
         p_last = static_cast<int>((static_cast<int64_t>(ts + ntb) * P_g - 1) / Nt);
     }
@@ -267,50 +269,71 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
         const int hi = static_cast<int>((static_cast<int64_t>(p + 1) * Nt) / P_g);
         return max(lo, ts) < min(hi, ts + ntb);
     };
-    for (int p = p_first; p <= p_last; ++p) {
-        if (!live(p)) continue;
-        const float2 ml = ml_part[(seg0 + p) * 128 + r];
-        if (ml.x == -CUDART_INF_F) continue;
-        const float Mn = fmaxf(M, ml.x);
-        z = z * exp2f(M - Mn) + ml.y * exp2f(ml.x - Mn);
-        M = Mn;
-    }
+    float M = -CUDART_INF_F, z = 0.f;
     float acc[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-    const int cg0 = 32 * qtr + 8 * k;
-    for (int p = p_first; p <= p_last; ++p) {
+    const int cg0 = 8 * slice;  // column groups 8 slice .. 8 slice + 7 = columns 32 slice .. + 31
+    for (int p = p_first + k; p <= p_last; p += kMergeSplit) {
         if (!live(p)) continue;
-        const float mp = ml_part[(seg0 + p) * 128 + r].x;
-        if (mp == -CUDART_INF_F) continue;
-        const float w = exp2f(mp - M);
-        // segment partials: [column group of 4][128 rows] x float4
+        // segment partials: [column group of 4][128 rows] x float4; the loads go out before the (m, l) test
         const float4* src = reinterpret_cast<const float4*>(o_part) + ((seg0 + p) * 128 + cg0) * 128 + r;
         float4 v[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = src[i * 128];
+        const float2 ml = ml_part[(seg0 + p) * 128 + r];
+        if (ml.x == -CUDART_INF_F) continue;
+        const float Mn = fmaxf(M, ml.x);
+        const float sc = exp2f(M - Mn), w = exp2f(ml.x - Mn);
+        z = z * sc + ml.y * w;
+        M = Mn;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            acc[4 * i] = fmaf(w, v[i].x, acc[4 * i]);
-            acc[4 * i + 1] = fmaf(w, v[i].y, acc[4 * i + 1]);
-            acc[4 * i + 2] = fmaf(w, v[i].z, acc[4 * i + 2]);
-            acc[4 * i + 3] = fmaf(w, v[i].w, acc[4 * i + 3]);
+            acc[4 * i] = fmaf(w, v[i].x, acc[4 * i] * sc);
+            acc[4 * i + 1] = fmaf(w, v[i].y, acc[4 * i + 1] * sc);
+            acc[4 * i + 2] = fmaf(w, v[i].z, acc[4 * i + 2] * sc);
+            acc[4 * i + 3] = fmaf(w, v[i].w, acc[4 * i + 3] * sc);
         }
     }
+    // combine the row's four partial merges (lanes 4 (r % 8) + 0..3)
+    float Mr = M;
+#pragma unroll
+    for (int o = 1; o < kMergeSplit; o <<= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
+    const float sc = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mr);
+    z *= sc;
+#pragma unroll
+    for (int o = 1; o < kMergeSplit; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        float a = acc[i] * sc;
+#pragma unroll
+        for (int o = 1; o < kMergeSplit; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        acc[i] = a;
+    }
+    if (!row_ok) return;
+    const int j = rr / H, h = rr % H;
+    const int t = b * n_q + j;
+    const int T = B * n_q;
     const float inv = (z > 0.f) ? 1.f / z : 0.f;
-    // columns 4 cg0 .. 4 cg0 + 31 = chunk (4 cg0) / 64, units 4 (k & 1) .. + 3
-    const int c = (4 * cg0) >> 6, u0 = 4 * (k & 1);
+    // columns 32 slice .. + 31 = chunk slice / 2, units 4 (slice & 1) .. + 3; thread k writes unit k
+    const int c = slice >> 1, u = 4 * (slice & 1) + k;
+    uint4 y;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        uint4 y;
-        y.x = pack_bf16x2(acc[8 * q] * inv, acc[8 * q + 1] * inv);
-        y.y = pack_bf16x2(acc[8 * q + 2] * inv, acc[8 * q + 3] * inv);
-        y.z = pack_bf16x2(acc[8 * q + 4] * inv, acc[8 * q + 5] * inv);
-        y.w = pack_bf16x2(acc[8 * q + 6] * inv, acc[8 * q + 7] * inv);
-        *reinterpret_cast<uint4*>(olat + olat_offset(T, h, t, c, u0 + q)) = y;
+        // thread k keeps the 16 bytes of columns 8 k .. 8 k + 7 of the slice
+        const float a0 = acc[8 * q] * inv, a1 = acc[8 * q + 1] * inv, a2 = acc[8 * q + 2] * inv,
+                    a3 = acc[8 * q + 3] * inv, a4 = acc[8 * q + 4] * inv, a5 = acc[8 * q + 5] * inv,
+                    a6 = acc[8 * q + 6] * inv, a7 = acc[8 * q + 7] * inv;
+        if (q == k) {
+            y.x = pack_bf16x2(a0, a1);
+            y.y = pack_bf16x2(a2, a3);
+            y.z = pack_bf16x2(a4, a5);
+            y.w = pack_bf16x2(a6, a7);
+        }
     }
-    if (qtr == 0 && k == 0 && lse_out)
-        lse_out[static_cast<int64_t>(t) * H + h] = (z > 0.f) ? (M + log2f(z)) * 0.69314718055994530942f : -CUDART_INF_F;
+    *reinterpret_cast<uint4*>(olat + olat_offset(T, h, t, c, u)) = y;
+    if (slice == 0 && k == 0 && lse_out)
+        lse_out[static_cast<int64_t>(t) * H + h] = (z > 0.f) ? (Mr + log2f(z)) * 0.69314718055994530942f : -CUDART_INF_F;
 }
 
 // ------------------------------------------------------------------ up-projection
@@ -477,7 +500,7 @@ cudaError_t launch_merge(const float* o_part, const float2* ml_part, const int32
                          cudaStream_t stream) {
     (void)dev_status;
     const int G = (n_q * H + 127) / 128;
-    const dim3 grid(4, B, G);
+    const dim3 grid(proj::kMergeSlices, B, G);
     return proj::launch_pdl(proj::merge_kernel, grid, proj::kMergeThreads, 0, stream, o_part, ml_part, kv_len,
                             max_blocks, B, n_q, H, P_g, slots, olat, lse_out);
 }
