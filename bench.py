@@ -410,11 +410,11 @@ def make_timer(torch, flush):
     return time_graph
 
 
-def measure_query_up(torch, mla, cfg, dev, time_graph, n, peaks, d_cq):
-    """Time mla_query_up (c^Q [T, d_c'] -> q^C, q^R) alone, as a CUDA graph after an L2 flush.
-
-    It is the step before absorb_q when queries are compressed, and is not part of the step above.
-    Algorithmic bytes: the weights H*192*d_c'*2, the c^Q rows in and q^C, q^R out.
+def measure_query_up(torch, mla, cfg, dev, time_graph, n, peaks, d_cq, W_UK=None):
+    """Time the compressed-query side alone, each as a CUDA graph after an L2 flush: mla_query_up
+    (c^Q [T, d_c'] -> q^C, q^R) and, with W_UK, mla_query_absorb (c^Q -> the absorbed query in one launch,
+    which replaces mla_query_up + mla_absorb_q).  Neither is part of the step (its queries arrive as q^C, q^R).
+    Algorithmic bytes: the weights read once, c^Q in, the outputs out.
     """
     cq, wuq, wqr = mi.compressed_queries(cfg, d_cq)
 
@@ -426,25 +426,39 @@ def measure_query_up(torch, mla, cfg, dev, time_graph, n, peaks, d_cq):
     qn = torch.empty((T, H, mi.D_H), dtype=torch.bfloat16, device=dev)
     qr = torch.empty((T, H, mi.D_R), dtype=torch.bfloat16, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    run = lambda: mla.query_up(cq_d, wuq_d, wqr_d, q_nope=qn, q_rope=qr, dev_status=status)
-    for _ in range(3):
-        run()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, capture_error_mode="relaxed"):
-        run()
-    torch.cuda.synchronize()
-    ms = time_graph(g, n)
-    torch.cuda.synchronize()
-    del g
+
+    def timed(run):
+        for _ in range(3):
+            run()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            run()
+        torch.cuda.synchronize()
+        us = 1e3 * statistics.mean(time_graph(g, n))
+        torch.cuda.synchronize()
+        del g
+        return us
+
+    def line(kernel, us, nbytes, **extra):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        return {"kernel": kernel, "d_cq": d_cq, "T": T, "H": H, "launches": n, "us_per_launch": round(us, 3),
+                "algorithmic_bytes": nbytes, "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), **extra}
+
+    us = timed(lambda: mla.query_up(cq_d, wuq_d, wqr_d, q_nope=qn, q_rope=qr, dev_status=status))
+    nbytes = H * (mi.D_H + mi.D_R) * d_cq * 2 + T * d_cq * 2 + T * H * (mi.D_H + mi.D_R) * 2
+    res = line("mla_query_up", us, nbytes, note="timed alone, L2 flushed before each launch; not part of the step")
+    if W_UK is not None:
+        pos = torch.arange(T, dtype=torch.int32, device=dev)
+        tab = mla.rope_table(max(T, 1), cfg.rope_base, dev)
+        qa = torch.empty((T, H, mi.D_ROW), dtype=torch.bfloat16, device=dev)
+        us = timed(lambda: mla.query_absorb(cq_d, wuq_d, wqr_d, W_UK, pos, tab, q_out=qa, dev_status=status))
+        nbytes = (H * (mi.D_H + mi.D_R) * d_cq * 2 + H * mi.D_H * mi.D_C * 2 + T * d_cq * 2 + T * H * mi.D_ROW * 2)
+        res["fused"] = line("mla_query_absorb", us, nbytes,
+                            note="c^Q -> absorbed query in one launch (= mla_query_up + mla_absorb_q)")
     if int(status.item()) != 0:
         return {"error": "device status " + mla.device_status_string(int(status.item()))}
-    nbytes = H * (mi.D_H + mi.D_R) * d_cq * 2 + T * d_cq * 2 + T * H * (mi.D_H + mi.D_R) * 2
-    us = 1e3 * statistics.mean(ms)
-    gbs = nbytes / (us * 1e-6) / 1e9
-    return {"kernel": "mla_query_up", "d_cq": d_cq, "T": T, "H": H, "launches": n, "us_per_launch": round(us, 3),
-            "algorithmic_bytes": nbytes, "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-            "note": "timed alone, L2 flushed before each launch; not part of the step"}
+    return res
 
 
 def prefill_flops(L: int, n: int, H: int) -> dict:
@@ -619,7 +633,7 @@ def measure_workload(torch, mla, dist, cfg, dev, args, flush, sampler=None, head
     if headline and dist.world == 1 and not args.no_query_up:
         try:
             res["query_up"] = measure_query_up(torch, mla, cfg, dev, time_graph, min(args.steps, 1000), peaks,
-                                               args.query_rank)
+                                               args.query_rank, W_UK=st["W_UK"])
         except Exception as e:  # reported in the line; the step's numbers above stand on their own
             res["query_up"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     del st

@@ -16,8 +16,9 @@
  *   - The same explainer, section 2.2.1.2: queries are compressed too, to c^Q,
  *     and up-projected (mla_query_up produces q^C and q^R from c^Q).
  *
- * Entry points, in the order a decode step uses them: mla_query_up (when
- * queries are compressed), mla_absorb_q, mla_append_cache, mla_decode (=
+ * Entry points, in the order a decode step uses them: mla_query_absorb (when
+ * queries are compressed; = mla_query_up + mla_absorb_q in one launch) or
+ * mla_absorb_q, mla_append_cache, mla_decode (=
  * mla_decode_attend + mla_decode_finish; mla_decode_static without a
  * workspace), with mla_decode_cudacore + mla_splitkv_combine as an
  * independent CUDA-core path of the same decode.  Long prefill chunks use
@@ -155,6 +156,30 @@ mla_status mla_absorb_q(const void* q_nope, const void* q_rope, const int32_t* p
  */
 mla_status mla_query_up(const void* c_q, const void* W_UQ, const void* W_QR, int T, int H, int d_cq,
                         void* q_nope, void* q_rope, int32_t* dev_status, mla_stream stream);
+
+/*
+ * mla_query_absorb -- mla_query_up and mla_absorb_q in one launch: from the
+ * compressed query c^Q straight to the absorbed query.
+ * (MLA explainer 2.2.1.2 and 2.2.2: q^C = W^UQ c^Q and the per-head q^R;
+ *  "两张账" page, "第一张账": W^UK absorbed into the query side.)
+ *   c_q     bf16 [T, d_cq]         compressed queries c^Q
+ *   W_UQ    bf16 [H, 128, d_cq]    W_QR bf16 [H, 64, d_cq]    W_UK bf16 [H, 128, 512]
+ *   pos     int32 [T] or NULL      position of query row t (NULL: q^R is not rotated)
+ *   q_out   bf16 [T, H, 576]       [ (W^UK_h)^T q^C[t, h] (512) | R_pos q^R[t, h] (64) ]
+ * q^C and q^R are rounded to bf16 exactly as mla_query_up stores them, and the
+ * rest is mla_absorb_q's arithmetic, so q_out is bit for bit the output of
+ * mla_query_up followed by mla_absorb_q; q^C never leaves the SM (it goes from
+ * tensor memory to shared memory as the operand of the absorption).  The
+ * order of operations is kept: no precomposed (W^UK_h)^T W^UQ_h is formed.
+ * Sizes: 1 <= H <= 128, d_cq a multiple of 64 in [64, 16384], T >= 0 (T = 0
+ * launches nothing).  Errors: as mla_query_up and mla_absorb_q (before any
+ * launch); a position outside the RoPE table sets MLA_DEVERR_POS_RANGE and that
+ * row's RoPE part is left unwritten; an expired bounded wait sets
+ * MLA_DEVERR_TIMEOUT.  Launched with programmatic stream serialization.
+ */
+mla_status mla_query_absorb(const void* c_q, const void* W_UQ, const void* W_QR, const void* W_UK,
+                            const int32_t* pos, const float* rope_table, int64_t rope_len, int T,
+                            int H, int d_cq, void* q_out, int32_t* dev_status, mla_stream stream);
 
 /*
  * mla_append_cache -- write T new tokens into the paged latent cache.

@@ -35,6 +35,7 @@ _SIGS = {
     "mla_rope_table_fill": ([_p, _i64, _f64], _i32),
     "mla_absorb_q": ([_p, _p, _p, _p, _p, _i64, _i32, _i32, _p, _p, _p], _i32),
     "mla_query_up": ([_p, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p], _i32),
+    "mla_query_absorb": ([_p, _p, _p, _p, _p, _p, _i64, _i32, _i32, _i32, _p, _p, _p], _i32),
     "mla_append_cache": ([_p, _i64, _p, _i32, _i32, _p, _p, _p, _p, _p, _i64, _i32, _p, _p], _i32),
     "mla_decode_workspace_bytes": ([_i32, _i32, _i32, _i32], _sz),
     "mla_decode": ([_p, _p, _i64, _p, _i32, _p, _p, _i32, _i32, _i32, _f32, _i32, _p, _sz, _p, _p, _p, _p], _i32),
@@ -126,6 +127,22 @@ def query_up(c_q, W_UQ, W_QR, q_nope=None, q_rope=None, dev_status=None, stream=
         _ptr(q_nope, torch.bfloat16, (T, H, D_H), "q_nope"), _ptr(q_rope, torch.bfloat16, (T, H, D_R), "q_rope"),
         _ptr(dev_status, torch.int32, None, "dev_status"), _stream(stream)))
     return q_nope, q_rope
+
+
+def query_absorb(c_q, W_UQ, W_QR, W_UK, pos, rope_tab, q_out=None, dev_status=None, stream=None):
+    """c^Q [T, d_cq] -> q_out bf16 [T, H, 576] = [(W^UK_h)^T (W^UQ_h c^Q) | R_pos (W^QR_h c^Q)] in one launch."""
+    T, d_cq = c_q.shape
+    H = W_UQ.shape[0]
+    if q_out is None:
+        q_out = torch.empty((T, H, D_ROW), dtype=torch.bfloat16, device=c_q.device)
+    _check(lib.mla_query_absorb(
+        _ptr(c_q, torch.bfloat16, (T, d_cq), "c_q"), _ptr(W_UQ, torch.bfloat16, (H, D_H, d_cq), "W_UQ"),
+        _ptr(W_QR, torch.bfloat16, (H, D_R, d_cq), "W_QR"), _ptr(W_UK, torch.bfloat16, (H, D_H, D_C), "W_UK"),
+        _ptr(pos, torch.int32, (T,), "pos"), _ptr(rope_tab, torch.float32, None, "rope_table"),
+        0 if rope_tab is None else rope_tab.shape[0], T, H, d_cq,
+        _ptr(q_out, torch.bfloat16, (T, H, D_ROW), "q_out"), _ptr(dev_status, torch.int32, None, "dev_status"),
+        _stream(stream)))
+    return q_out
 
 
 def new_cache(cap_blocks: int, device="cuda") -> torch.Tensor:

@@ -150,6 +150,21 @@ mla_status mla_query_up(const void* c_q, const void* W_UQ, const void* W_QR, int
                                        static_cast<uint16_t*>(q_rope), dev_status, static_cast<cudaStream_t>(stream)));
 }
 
+mla_status mla_query_absorb(const void* c_q, const void* W_UQ, const void* W_QR, const void* W_UK, const int32_t* pos,
+                            const float* rope_table, int64_t rope_len, int T, int H, int d_cq, void* q_out,
+                            int32_t* dev_status, mla_stream stream) {
+    if (T < 0 || rope_len < 0) return MLA_ERR_INVALID_ARG;
+    if (H < 1 || H > kMaxHeads || d_cq < 64 || d_cq > 16384 || d_cq % 64 != 0) return MLA_ERR_UNSUPPORTED_SHAPE;
+    if (T == 0) return MLA_OK;
+    if (!c_q || !W_UQ || !W_QR || !W_UK || !q_out || (pos && !rope_table)) return MLA_ERR_INVALID_ARG;
+    if (!aligned16(c_q) || !aligned16(W_UQ) || !aligned16(W_QR) || !aligned16(W_UK) || !aligned16(q_out))
+        return MLA_ERR_INVALID_ARG;
+    return cuda_status(launch_query_absorb(static_cast<const uint16_t*>(c_q), static_cast<const uint16_t*>(W_UQ),
+                                           static_cast<const uint16_t*>(W_QR), static_cast<const uint16_t*>(W_UK), pos,
+                                           rope_table, rope_len, T, H, d_cq, static_cast<uint16_t*>(q_out),
+                                           dev_status, static_cast<cudaStream_t>(stream)));
+}
+
 mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int32_t* block_table, int num_seqs,
                             int max_blocks, const int32_t* seq_idx, const int32_t* pos, const void* c_kv, const void* k_rope,
                             const float* rope_table, int64_t rope_len, int T, int32_t* dev_status,

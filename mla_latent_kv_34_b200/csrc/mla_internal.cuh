@@ -70,6 +70,11 @@ cudaError_t launch_absorb_tc(const uint16_t* q_nope, const uint16_t* q_rope, con
 cudaError_t launch_query_up(const uint16_t* c_q, const uint16_t* W_UQ, const uint16_t* W_QR, int T, int H, int d_cq,
                             uint16_t* q_nope, uint16_t* q_rope, int32_t* dev_status, cudaStream_t stream);
 
+// The compressed-query up-projections fused with the absorption of W^UK (query_absorb.cu).
+cudaError_t launch_query_absorb(const uint16_t* c_q, const uint16_t* W_UQ, const uint16_t* W_QR, const uint16_t* W_UK,
+                                const int32_t* pos, const float* rope_table, int64_t rope_len, int T, int H, int d_cq,
+                                uint16_t* q_out, int32_t* dev_status, cudaStream_t stream);
+
 // Naive-form attention for long prefill chunks (prefill_naive.cu).
 size_t prefill_rows_bytes(int L, int H);
 cudaError_t launch_prefill_naive(const uint16_t* q_nope, const uint16_t* q_rope, const float* rope_table,

@@ -106,6 +106,12 @@ def test_host_validation_rejects_bad_arguments(mla):
     assert pre(scale=0.0) == 1
     assert pre(ws_bytes=100) == 4
     assert L.mla_prefill_workspace_bytes(300, 16) == 2 * 300 * 16 * 128 * 2
+    # fused query side: empty, bad d_cq, bad H, null W^UK, rope table missing with positions
+    assert L.mla_query_absorb(None, None, None, None, None, None, 0, 0, 16, 1536, None, None, None) == 0
+    assert L.mla_query_absorb(fake, fake, fake, fake, None, None, 0, 4, 16, 100, fake, None, None) == 2
+    assert L.mla_query_absorb(fake, fake, fake, fake, None, None, 0, 4, 129, 1536, fake, None, None) == 2
+    assert L.mla_query_absorb(fake, fake, fake, None, None, None, 0, 4, 16, 1536, fake, None, None) == 1
+    assert L.mla_query_absorb(fake, fake, fake, fake, fake, None, 0, 4, 16, 1536, fake, None, None) == 1
     # query up-projection: empty, d_cq not a multiple of 64, no heads, null input
     assert L.mla_query_up(None, None, None, 0, 16, 1536, None, None, None, None) == 0
     assert L.mla_query_up(fake, fake, fake, 4, 16, 100, fake, fake, None, None) == 2

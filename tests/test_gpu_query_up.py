@@ -75,3 +75,43 @@ def test_query_up_chain_to_decode(H):
                                     scale=cfg.scale, base=cfg.rope_base)
         assert np.all(np.abs(got[b] - ref) <= 1e-2 + 1e-2 * np.abs(ref)), f"sequence {b}"
         assert np.linalg.norm(got[b] - ref) / np.linalg.norm(ref) < 1e-2
+
+
+@pytest.mark.parametrize("T,nh,d_cq", [(1, 1, 64), (17, 16, 1536), (32, 128, 1536), (130, 3, 576),
+                                       (200, 8, 128), (256, 128, 1536), (64, 5, 192)])
+def test_query_absorb_is_query_up_then_absorb(H, T, nh, d_cq):
+    """The fused c^Q -> q_abs call equals mla_query_up followed by mla_absorb_q bit for bit, and the
+    oracle's fp64 chain W^UK^T (W^UQ c^Q), R_pos (W^QR c^Q) within one bf16 rounding of each step."""
+    import mla_latent_kv_34_b200 as mla
+    cfg = mi.MLAConfig("qabs", B=T, H=nh, n_q=1, L=1, seed=6000 + T + nh + d_cq)
+    cq, wuq, wqr = mi.compressed_queries(cfg, d_cq)
+    wuk = mi.weights(cfg, "uk")
+    dev = "cuda"
+    pos = ((np.arange(T) * 7919 + 3) % 131072).astype(np.int32)
+    tab = mla.rope_table(131072, 10000.0, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    cq_d, wuq_d, wqr_d, wuk_d = (H.to_dev_bf16(x, dev) for x in (cq, wuq, wqr, wuk))
+    pos_d = torch.from_numpy(pos).to(dev)
+    fused = mla.query_absorb(cq_d, wuq_d, wqr_d, wuk_d, pos_d, tab, dev_status=status)
+    qn, qr = mla.query_up(cq_d, wuq_d, wqr_d, dev_status=status)
+    two = mla.absorb_q(qn, qr, pos_d, wuk_d, tab, dev_status=status)
+    unrot = mla.query_absorb(cq_d, wuq_d, wqr_d, wuk_d, None, tab, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(fused.view(torch.int16), two.view(torch.int16))
+    # pos = NULL: the RoPE part is q^R as rounded, not rotated
+    assert torch.equal(unrot[..., 512:].view(torch.int16), qr.view(torch.int16))
+    f = mi.bf16_bits_to_f64
+    ref_n, ref_r = on.query_up(f(cq), f(wuq), f(wqr))
+    ref_abs = on.absorb_query(ref_n, f(wuk))
+    ref_pe = on.rope(ref_r, pos[:, None])
+    got = fused.float().cpu().numpy()
+    # Rigorous bounds: q^C (and q^R) are rounded to bf16 once (|delta_i| <= 2^-9 |q_i|); through W^UK that
+    # is at most 2^-9 sum_i |W^UK[i, c]| |q^C_i|; the output is rounded once more (<= 2^-9 |value|, taken
+    # as 2^-8 |ref| to cover the first error's share of the value); fp32 sums add far less than 1e-5.
+    prop = 2.0 ** -9 * np.einsum("hic,thi->thc", np.abs(f(wuk)), np.abs(ref_n))
+    assert np.all(np.abs(got[..., :512] - ref_abs) <= prop + 2.0 ** -8 * np.abs(ref_abs) + 1e-5)
+    # RoPE part: a rotation of the rounded pair, so the pair's rounding error stays within 2^-9 (|x0| + |x1|)
+    pair = np.abs(ref_r[..., 0::2]) + np.abs(ref_r[..., 1::2])
+    prop_r = 2.0 ** -9 * np.repeat(pair, 2, axis=-1)
+    assert np.all(np.abs(got[..., 512:] - ref_pe) <= prop_r + 2.0 ** -8 * np.abs(ref_pe) + 1e-5)
