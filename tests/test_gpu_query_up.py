@@ -106,12 +106,13 @@ def test_query_absorb_is_query_up_then_absorb(H, T, nh, d_cq):
     ref_abs = on.absorb_query(ref_n, f(wuk))
     ref_pe = on.rope(ref_r, pos[:, None])
     got = fused.float().cpu().numpy()
-    # Rigorous bounds: q^C (and q^R) are rounded to bf16 once (|delta_i| <= 2^-9 |q_i|); through W^UK that
-    # is at most 2^-9 sum_i |W^UK[i, c]| |q^C_i|; the output is rounded once more (<= 2^-9 |value|, taken
-    # as 2^-8 |ref| to cover the first error's share of the value); fp32 sums add far less than 1e-5.
-    prop = 2.0 ** -9 * np.einsum("hic,thi->thc", np.abs(f(wuk)), np.abs(ref_n))
-    assert np.all(np.abs(got[..., :512] - ref_abs) <= prop + 2.0 ** -8 * np.abs(ref_abs) + 1e-5)
-    # RoPE part: a rotation of the rounded pair, so the pair's rounding error stays within 2^-9 (|x0| + |x1|)
+    # Rigorous bounds: q^C (and q^R) are rounded to bf16 once, a relative error of at most u = 2^-8 (bf16
+    # keeps 8 significant bits); through W^UK that is at most u sum_i |W^UK[i, c]| |q^C_i|; the output is
+    # rounded once more (at most u |value|, taken as u (1 + 2^-6) |ref|); fp32 sums add far less than 1e-5.
+    u = 2.0 ** -8
+    prop = u * np.einsum("hic,thi->thc", np.abs(f(wuk)), np.abs(ref_n))
+    assert np.all(np.abs(got[..., :512] - ref_abs) <= prop + u * (1 + 2 ** -6) * np.abs(ref_abs) + 1e-5)
+    # RoPE part: a rotation of the rounded pair, so the pair's rounding error stays within u (|x0| + |x1|)
     pair = np.abs(ref_r[..., 0::2]) + np.abs(ref_r[..., 1::2])
-    prop_r = 2.0 ** -9 * np.repeat(pair, 2, axis=-1)
-    assert np.all(np.abs(got[..., 512:] - ref_pe) <= prop_r + 2.0 ** -8 * np.abs(ref_pe) + 1e-5)
+    prop_r = u * np.repeat(pair, 2, axis=-1)
+    assert np.all(np.abs(got[..., 512:] - ref_pe) <= prop_r + u * (1 + 2 ** -6) * np.abs(ref_pe) + 1e-5)
