@@ -202,8 +202,6 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
 
 // ------------------------------------------------------------------ merge
 
-constexpr int kMergeSplit = 4;                       // threads per row, each taking every 4th piece
-constexpr int kMergeThreads = 128 * kMergeSplit;     // a warp = 8 rows x 4 threads
 constexpr int kMergeSlices = 16;    // a CTA merges 32 of the 512 latent columns (8 column groups of 4)
 
 // Byte offset of row t of head h, latent unit (chunk c, unit u) in the o_lat tiles: per head, the rows
@@ -216,17 +214,21 @@ __device__ __forceinline__ int64_t olat_offset(int T, int h, int t, int c, int u
     return (static_cast<int64_t>(h) * Tp + 64 * tb) * 1024 + c * rows * 128 + swz(i, u);
 }
 
-// One CTA per (32-column slice, sequence, row group).  Row r of the group is merged by four threads,
-// lanes 4 (r % 8) .. + 3 of warp r / 8, each over every fourth piece of the sequence with its own running
-// maximum; the four partial results are combined with warp shuffles.  A thread's loads of one piece are
-// eight 16-byte column groups of its row (the attend kernel's [column group][row] order).
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(
+// One CTA per (32-column slice, sequence, row group).  Row r of the group is merged by kSplit threads
+// (neighbouring lanes), each over every kSplit-th piece of the sequence with its own running maximum; their
+// partial results are combined with warp shuffles.  kSplit follows the expected pieces per sequence (1 when
+// sequences outnumber the CTA pairs, up to 4 for a few long sequences cut into many pieces).  A thread's
+// loads of one piece are eight 16-byte column groups of its row (the attend kernel's [column group][row]
+// order).
+template <int kSplit>
+__global__ void __launch_bounds__(128 * kSplit) merge_kernel(
     const float* __restrict__ o_part, const float2* __restrict__ ml_part, const int32_t* __restrict__ kv_len,
     int max_blocks, int B, int n_q, int H, int P_g, int slots, uint8_t* __restrict__ olat, float* __restrict__ lse_out) {
+    constexpr int kMergeThreads = 128 * kSplit;
     __shared__ int red[2][kMergeThreads / 32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
-    const int r = 8 * warp + (lane >> 2), k = lane & 3;
+    const int r = tid / kSplit, k = tid % kSplit;
     grid_dependency_wait();  // the pieces come from the attend kernel
     grid_dependents_launch();
     // tiles of all sequences (the attend kernel's range split depends on the total) and before b
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] = 0.f;
     const int cg0 = 8 * slice;  // column groups 8 slice .. 8 slice + 7 = columns 32 slice .. + 31
-    for (int p = p_first + k; p <= p_last; p += kMergeSplit) {
+    for (int p = p_first + k; p <= p_last; p += kSplit) {
         if (!live(p)) continue;
         // segment partials: [column group of 4][128 rows] x float4; the loads go out before the (m, l) test
         const float4* src = reinterpret_cast<const float4*>(o_part) + ((seg0 + p) * 128 + cg0) * 128 + r;
@@ -295,19 +297,19 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
             acc[4 * i + 3] = fmaf(w, v[i].w, acc[4 * i + 3] * sc);
         }
     }
-    // combine the row's four partial merges (lanes 4 (r % 8) + 0..3)
+    // combine the row's kSplit partial merges (neighbouring lanes)
     float Mr = M;
 #pragma unroll
-    for (int o = 1; o < kMergeSplit; o <<= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
+    for (int o = 1; o < kSplit; o <<= 1) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, o));
     const float sc = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mr);
     z *= sc;
 #pragma unroll
-    for (int o = 1; o < kMergeSplit; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    for (int o = 1; o < kSplit; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
         float a = acc[i] * sc;
 #pragma unroll
-        for (int o = 1; o < kMergeSplit; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        for (int o = 1; o < kSplit; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
         acc[i] = a;
     }
     if (!row_ok) return;
@@ -315,23 +317,19 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const int t = b * n_q + j;
     const int T = B * n_q;
     const float inv = (z > 0.f) ? 1.f / z : 0.f;
-    // columns 32 slice .. + 31 = chunk slice / 2, units 4 (slice & 1) .. + 3; thread k writes unit k
-    const int c = slice >> 1, u = 4 * (slice & 1) + k;
-    uint4 y;
+    // columns 32 slice .. + 31 = chunk slice / 2, units 4 (slice & 1) .. + 3; thread k writes the units
+    // q with q % kSplit == k (16 bytes = columns 8 q .. 8 q + 7 of the slice)
+    const int c = slice >> 1;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        // thread k keeps the 16 bytes of columns 8 k .. 8 k + 7 of the slice
-        const float a0 = acc[8 * q] * inv, a1 = acc[8 * q + 1] * inv, a2 = acc[8 * q + 2] * inv,
-                    a3 = acc[8 * q + 3] * inv, a4 = acc[8 * q + 4] * inv, a5 = acc[8 * q + 5] * inv,
-                    a6 = acc[8 * q + 6] * inv, a7 = acc[8 * q + 7] * inv;
-        if (q == k) {
-            y.x = pack_bf16x2(a0, a1);
-            y.y = pack_bf16x2(a2, a3);
-            y.z = pack_bf16x2(a4, a5);
-            y.w = pack_bf16x2(a6, a7);
-        }
+        if (q % kSplit != k) continue;
+        uint4 y;
+        y.x = pack_bf16x2(acc[8 * q] * inv, acc[8 * q + 1] * inv);
+        y.y = pack_bf16x2(acc[8 * q + 2] * inv, acc[8 * q + 3] * inv);
+        y.z = pack_bf16x2(acc[8 * q + 4] * inv, acc[8 * q + 5] * inv);
+        y.w = pack_bf16x2(acc[8 * q + 6] * inv, acc[8 * q + 7] * inv);
+        *reinterpret_cast<uint4*>(olat + olat_offset(T, h, t, c, 4 * (slice & 1) + q)) = y;
     }
-    *reinterpret_cast<uint4*>(olat + olat_offset(T, h, t, c, u)) = y;
     if (slice == 0 && k == 0 && lse_out)
         lse_out[static_cast<int64_t>(t) * H + h] = (z > 0.f) ? (Mr + log2f(z)) * 0.69314718055994530942f : -CUDART_INF_F;
 }
@@ -501,8 +499,16 @@ cudaError_t launch_merge(const float* o_part, const float2* ml_part, const int32
     (void)dev_status;
     const int G = (n_q * H + 127) / 128;
     const dim3 grid(proj::kMergeSlices, B, G);
-    return proj::launch_pdl(proj::merge_kernel, grid, proj::kMergeThreads, 0, stream, o_part, ml_part, kv_len,
-                            max_blocks, B, n_q, H, P_g, slots, olat, lse_out);
+    // pieces per sequence ~ 1 + P_g / B: one thread per row when sequences outnumber the pairs
+    const int per = P_g / (B > 0 ? B : 1);
+    if (per >= 4)
+        return proj::launch_pdl(proj::merge_kernel<4>, grid, 512, 0, stream, o_part, ml_part, kv_len, max_blocks, B,
+                                n_q, H, P_g, slots, olat, lse_out);
+    if (per >= 1)
+        return proj::launch_pdl(proj::merge_kernel<2>, grid, 256, 0, stream, o_part, ml_part, kv_len, max_blocks, B,
+                                n_q, H, P_g, slots, olat, lse_out);
+    return proj::launch_pdl(proj::merge_kernel<1>, grid, 128, 0, stream, o_part, ml_part, kv_len, max_blocks, B, n_q,
+                            H, P_g, slots, olat, lse_out);
 }
 
 cudaError_t launch_upproj(const uint8_t* olat, const uint16_t* W_UV, int T, int H, uint16_t* out, int32_t* dev_status,

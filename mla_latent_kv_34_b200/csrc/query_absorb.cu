@@ -11,15 +11,16 @@
 // q^C never leaves the SM: it goes from TMEM to shared memory as the B operand of the absorption.
 // The result is bit for bit the result of mla_query_up followed by mla_absorb_q.
 //
-// One CTA per (head, block of up to 64 query rows).
-//  stage 1: d_c' streams through two 64 KB shared-memory stages, two 64-column chunks per stage:
-//           W^UQ_h [128 x 128] (one 3-D TMA box), W^QR_h [64 x 128] (one box) and the c^Q rows
-//           [NT x 128] (one box).  Per 16-column step two MMAs: q^C into TMEM columns 0..NT-1 and,
-//           reading 128 rows from the W^QR chunk, q^R into lanes 0..63 of columns 64..64+NT-1 (the
-//           other 64 rows read whatever follows; their lanes are never used).
+// One CTA per (head, block of up to 128 query rows).
+//  stage 1: d_c' streams through four 40 KB shared-memory stages, one 64-column chunk per stage:
+//           W^UQ_h [128 x 64] and W^QR_h [64 x 64] land as one stacked [192 x 64] chunk, the c^Q rows
+//           [NT x 64] beside it (three TMA boxes).  Per 16-column step two M = 128 MMAs read the
+//           stacked chunk from row 0 (q^C into TMEM columns 0..NT-1) and from row 64 (lanes 64..127 are
+//           q^R, in columns 128..128+NT-1; the duplicated rows are ignored).
 //  stage 2: W^UK_h (eight [128 x 64] boxes, 128 KB) lands in the freed stages; the epilogue warps move
 //           q^C (bf16) into a swizzled [NT x 128] tile and rotate q^R; 32 MMAs (4 blocks of 128
-//           latent columns, M = 128, N = NT) form the absorbed query in TMEM columns 128..
+//           latent columns, M = 128, N = NT) then form the absorbed query in TMEM columns 0..4 NT - 1,
+//           which the consumed q^C / q^R accumulators no longer need.
 // Warps 0..3: epilogue; warp 4 lane 0: TMA; warp 5 lane 0: MMA.  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -33,18 +34,23 @@ using namespace sm100;
 namespace qab {
 
 constexpr int kThreads = 192;
-constexpr int kTokBlock = 64;                 // query rows per CTA (MMA N <= 64)
+constexpr int kTokBlock = 128;                // query rows per CTA (MMA N <= 128)
 constexpr int kChunkBytes = 128 * 128;        // [128 rows x 64 columns] bf16
-constexpr int kStageBytes = 65536;            // W^UQ 32 KB | W^QR 16 KB | c^Q <= 16 KB
-constexpr int kOffUq = 0, kOffQr = 32768, kOffCq = 49152;
-constexpr int kOffB2 = 2 * kStageBytes;       // q^C as the absorption's B operand: 2 x [NT x 64], 16 KB
-constexpr int kOffBar = kOffB2 + kTokBlock * 256;
+constexpr int kStages = 4;
+constexpr int kStageBytes = 40960;            // W^UQ 16 KB | W^QR 8 KB | c^Q <= 16 KB
+constexpr int kOffUq = 0, kOffQr = 16384, kOffCq = 24576;
+constexpr int kOffB2 = kStages * kStageBytes; // q^C as the absorption's B operand: 2 x [NT x 64], <= 32 KB
+constexpr int kOffRope = kOffB2 + kTokBlock * 256;  // (cos, sin) rows of the tile's query positions, <= 32 KB
+constexpr int kOffPos = kOffRope + kTokBlock * kDr * 4;  // positions of the tile's rows (-1: none / outside)
+constexpr int kOffBar = kOffPos + kTokBlock * 4;
 constexpr int kSmemBytes = kOffBar + 256;
-constexpr uint32_t kColC = 0, kColR = 64, kColAbs = 128;
+constexpr int kOutRowBytes = kDc * 2;         // the absorbed part of one output row, staged in the stages
+constexpr uint32_t kColC = 0, kColR = 128, kColAbs = 0;
+static_assert(kStages * kStageBytes >= 8 * kChunkBytes, "W^UK_h fits in the stages");
 constexpr uint64_t kLimitNs = 2000000000ull;
-static_assert(kOffB2 % 1024 == 0 && kOffCq % 1024 == 0, "swizzled operands 1024-aligned");
+static_assert(kOffB2 % 1024 == 0 && kOffCq % 1024 == 0 && kStageBytes % 1024 == 0, "swizzled operands 1024-aligned");
 
-enum { kBFull = 0, kBEmpty = 2, kBDone1 = 4, kBWFull = 5, kBQcReady = 6, kBDone2 = 7, kBCount = 8 };
+enum { kBFull = 0, kBEmpty = kStages, kBDone1 = 2 * kStages, kBWFull, kBQcReady, kBDone2, kBCount };
 
 __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
     const __grid_constant__ CUtensorMap uq_map, const __grid_constant__ CUtensorMap qr_map,
@@ -60,8 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
     const int h = blockIdx.x;
     const int t0 = blockIdx.y * kTokBlock;
     const int nt = min(kTokBlock, T - t0);
-    const int KC = d_cq / 64;       // 64-column chunks of d_c'
-    const int NS = (KC + 1) / 2;    // stages (an odd last chunk is paired with a zero-filled one)
+    const int KC = d_cq / 64;       // 64-column chunks of d_c', one per stage round
     volatile int never = 0;
     if ((sbase & 1023u) != 0) {
         if (tid == 0) report(dev_status, MLA_DEVERR_TIMEOUT);
@@ -78,6 +83,28 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     grid_dependency_wait();  // inputs may come from the previous kernel on the stream
+    int32_t* pos_s = reinterpret_cast<int32_t*>(smem + kOffPos);
+    float* rope_s = reinterpret_cast<float*>(smem + kOffRope);
+    if (warp < 4) {
+        // while stage 1 streams: the tile's positions and their (cos, sin) rows into shared memory
+        int32_t pp = -1;
+        if (tid < nt && pos) {
+            pp = pos[t0 + tid];
+            if (pp < 0 || pp >= rope_len) {
+                report(dev_status, MLA_DEVERR_POS_RANGE);
+                pp = -2;
+            }
+        }
+        pos_s[tid] = pp;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int i = tid; i < nt * (kDr / 4); i += 128) {
+            const int j = i / (kDr / 4), q = i % (kDr / 4);
+            const int32_t pj = pos_s[j];
+            if (pj >= 0)
+                reinterpret_cast<float4*>(rope_s)[j * (kDr / 4) + q] =
+                    reinterpret_cast<const float4*>(rope_table + static_cast<int64_t>(pj) * kDr)[q];
+        }
+    }
 
     if (warp == 4 && lane == 0) {
         // ---- TMA producer
@@ -85,23 +112,23 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
         prefetch_tmap(&qr_map);
         prefetch_tmap(&cq_map);
         prefetch_tmap(&uk_map);
-        const uint32_t tx = 32768u + 16384u + static_cast<uint32_t>(NT) * 256u;
+        const uint32_t tx = 16384u + 8192u + static_cast<uint32_t>(NT) * 128u;
         bool ok = true;
-        for (int ks = 0; ks < NS && ok; ++ks) {
-            const int s = ks & 1, n = ks >> 1;
+        for (int k = 0; k < KC && ok; ++k) {
+            const int s = k % kStages, n = k / kStages;
             if (n > 0 && !mbar_wait(&bars[kBEmpty + s], (n - 1) & 1, abort_flag, kLimitNs)) {
                 ok = false;
                 break;
             }
             const uint32_t st = sbase + s * kStageBytes;
             mbar_arrive_expect_tx(&bars[kBFull + s], tx);
-            tma_load_3d(st + kOffUq, &uq_map, 0, h * 128, 2 * ks, &bars[kBFull + s]);
-            tma_load_3d(st + kOffQr, &qr_map, 0, h * 64, 2 * ks, &bars[kBFull + s]);
-            tma_load_3d(st + kOffCq, &cq_map, 0, t0, 2 * ks, &bars[kBFull + s]);
+            tma_load_3d(st + kOffUq, &uq_map, 0, h * 128, k, &bars[kBFull + s]);
+            tma_load_3d(st + kOffQr, &qr_map, 0, h * 64, k, &bars[kBFull + s]);
+            tma_load_3d(st + kOffCq, &cq_map, 0, t0, k, &bars[kBFull + s]);
         }
-        // W^UK_h into both stages once their last stage-1 MMAs have completed
-        for (int s = 0; ok && s < 2 && s < NS; ++s) {
-            const int last = ((NS - 1 - s) >> 1);  // use index of stage s's final round
+        // W^UK_h into the stages once the last stage-1 MMAs of each have completed
+        for (int s = 0; ok && s < kStages && s < KC; ++s) {
+            const int last = (KC - 1 - s) / kStages;  // use index of stage s's final round
             ok = mbar_wait(&bars[kBEmpty + s], last & 1, abort_flag, kLimitNs);
         }
         if (ok) {
@@ -116,8 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
         // ---- MMA issuer
         bool ok = true;
         const uint32_t idesc1 = idesc_bf16_f32(128, NT, false, false);
-        for (int ks = 0; ks < NS; ++ks) {
-            const int s = ks & 1, n = ks >> 1;
+        for (int k = 0; k < KC; ++k) {
+            const int s = k % kStages, n = k / kStages;
             if (!mbar_wait(&bars[kBFull + s], n & 1, abort_flag, kLimitNs)) {
                 ok = false;
                 break;
@@ -125,16 +152,15 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
             tc_fence_after();
             const uint32_t st = sbase + s * kStageBytes;
 #pragma unroll
-            for (int kc = 0; kc < 2; ++kc)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ac = sdesc_sw128(st + kOffUq + kc * kChunkBytes + kk * 32, 16, 1024);
-                    const uint64_t ar = sdesc_sw128(st + kOffQr + kc * (kChunkBytes / 2) + kk * 32, 16, 1024);
-                    const uint64_t b = sdesc_sw128(st + kOffCq + kc * NT * 128 + kk * 32, 16, 1024);
-                    const uint32_t acc = (ks > 0 || kc > 0 || kk > 0) ? 1u : 0u;
-                    mma_ss(tmem + kColC, ac, b, idesc1, acc);
-                    mma_ss(tmem + kColR, ar, b, idesc1, acc);
-                }
+            for (int kk = 0; kk < 4; ++kk) {
+                // the stacked [192 x 64] chunk read from row 0 (W^UQ) and from row 64 (lanes 64..127: W^QR)
+                const uint64_t ac = sdesc_sw128(st + kOffUq + kk * 32, 16, 1024);
+                const uint64_t ar = sdesc_sw128(st + 64 * 128 + kk * 32, 16, 1024);
+                const uint64_t b = sdesc_sw128(st + kOffCq + kk * 32, 16, 1024);
+                const uint32_t acc = (k > 0 || kk > 0) ? 1u : 0u;
+                mma_ss(tmem + kColC, ac, b, idesc1, acc);
+                mma_ss(tmem + kColR, ar, b, idesc1, acc);
+            }
             mma_commit(smem_u32(&bars[kBEmpty + s]));
         }
         mma_commit(smem_u32(&bars[kBDone1]));
@@ -185,9 +211,11 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
                     }
                 }
             }
-            // q^R dims 0..63 (warps 0, 1): rounded to bf16, then rotated at the query position with the
-            // same fp32 arithmetic as mla_absorb_q; the pair (2i, 2i+1) sits in lanes (2i, 2i+1)
-            if (warp < 2) {
+            // q^R dims 0..63 = TMEM lanes 64..127 of its accumulator (warps 2, 3): rounded to bf16, then
+            // rotated at the query position with the same fp32 arithmetic as mla_absorb_q; the pair
+            // (2i, 2i+1) sits in neighbouring lanes
+            if (warp >= 2) {
+                const int dr = d - 64;  // dim of q^R
                 for (int j0 = 0; j0 < NT; j0 += 32) {
                     uint32_t v[32];
                     if (NT - j0 >= 32) tmem_ld32(t_lane + kColR + j0, v);
@@ -203,19 +231,17 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
                             uint16_t y = xb;
                             bool write = true;
                             if (pos) {
-                                const int32_t pp = pos[t];
-                                if (pp < 0 || pp >= rope_len) {
-                                    if (lane == 0) report(dev_status, MLA_DEVERR_POS_RANGE);
-                                    write = false;
+                                const int32_t pp = pos_s[j0 + j];
+                                if (pp < 0) {
+                                    write = false;  // reported when the positions were read
                                 } else {
-                                    const float2 cs =
-                                        reinterpret_cast<const float2*>(rope_table + static_cast<int64_t>(pp) * kDr)[d >> 1];
-                                    const float x0 = bf16_to_f32((d & 1) ? ob : xb), x1 = bf16_to_f32((d & 1) ? xb : ob);
-                                    y = (d & 1) ? f32_to_bf16_rne(__fadd_rn(__fmul_rn(x0, cs.y), __fmul_rn(x1, cs.x)))
-                                                : f32_to_bf16_rne(__fsub_rn(__fmul_rn(x0, cs.x), __fmul_rn(x1, cs.y)));
+                                    const float2 cs = reinterpret_cast<const float2*>(rope_s + (j0 + j) * kDr)[dr >> 1];
+                                    const float x0 = bf16_to_f32((dr & 1) ? ob : xb), x1 = bf16_to_f32((dr & 1) ? xb : ob);
+                                    y = (dr & 1) ? f32_to_bf16_rne(__fadd_rn(__fmul_rn(x0, cs.y), __fmul_rn(x1, cs.x)))
+                                                 : f32_to_bf16_rne(__fsub_rn(__fmul_rn(x0, cs.x), __fmul_rn(x1, cs.y)));
                                 }
                             }
-                            if (write) q_out[(static_cast<int64_t>(t) * H + h) * kRow + kDc + d] = y;
+                            if (write) q_out[(static_cast<int64_t>(t) * H + h) * kRow + kDc + dr] = y;
                         }
                     }
                 }
@@ -228,6 +254,9 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
         ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
         tc_fence_after();
         if (ok) {
+            // the MMAs are done with W^UK: stage the absorbed rows, bf16 [nt x 512] row-major, in the stages
+            // (a thread writes its latent column of 32 rows at a time: a warp store is 64 contiguous bytes)
+            uint8_t* stage_out = smem;
             for (int mb = 0; mb < 4; ++mb) {
                 const int c = 128 * mb + d;  // latent column of this TMEM lane in block mb
                 for (int j0 = 0; j0 < NT; j0 += 32) {
@@ -240,9 +269,17 @@ __global__ void __launch_bounds__(kThreads, 1) query_absorb_kernel(
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
                         if (j < jn)
-                            q_out[(static_cast<int64_t>(t0 + j0 + j) * H + h) * kRow + c] =
+                            *reinterpret_cast<uint16_t*>(stage_out + (j0 + j) * kOutRowBytes + 2 * c) =
                                 f32_to_bf16_rne(__uint_as_float(v[j]));
                 }
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            // then each output row's 1 KB goes out as 16-byte stores, consecutive threads on one row
+            for (int i = tid; i < nt * (kOutRowBytes / 16); i += 128) {
+                const int j = i / (kOutRowBytes / 16), q = i % (kOutRowBytes / 16);
+                *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(q_out) +
+                                          ((static_cast<int64_t>(t0 + j) * H + h) * kRow) * 2 + 16 * q) =
+                    *reinterpret_cast<const uint4*>(stage_out + j * kOutRowBytes + 16 * q);
             }
         } else if (lane == 0) {
             report(dev_status, MLA_DEVERR_TIMEOUT);
@@ -294,9 +331,9 @@ cudaError_t launch_query_absorb(const uint16_t* c_q, const uint16_t* W_UQ, const
                                 uint16_t* q_out, int32_t* dev_status, cudaStream_t stream) {
     const int NT = T >= qab::kTokBlock ? qab::kTokBlock : ((T + 15) & ~15);
     CUtensorMap uq, qr, cq, uk;
-    if (!qab::chunked_map(&uq, W_UQ, static_cast<uint64_t>(H) * 128, d_cq, 128, 2) ||
-        !qab::chunked_map(&qr, W_QR, static_cast<uint64_t>(H) * 64, d_cq, 64, 2) ||
-        !qab::chunked_map(&cq, c_q, static_cast<uint64_t>(T), d_cq, static_cast<uint32_t>(NT), 2) ||
+    if (!qab::chunked_map(&uq, W_UQ, static_cast<uint64_t>(H) * 128, d_cq, 128, 1) ||
+        !qab::chunked_map(&qr, W_QR, static_cast<uint64_t>(H) * 64, d_cq, 64, 1) ||
+        !qab::chunked_map(&cq, c_q, static_cast<uint64_t>(T), d_cq, static_cast<uint32_t>(NT), 1) ||
         !qab::chunked_map(&uk, W_UK, static_cast<uint64_t>(H) * 128, kDc, 128, 1))
         return cudaErrorNotSupported;
     cudaError_t e = cudaFuncSetAttribute(qab::query_absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
