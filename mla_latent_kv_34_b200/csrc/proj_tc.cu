@@ -14,13 +14,17 @@
 // absorb: one CTA per (128 latent columns, head, up to 64 query rows), so 4 CTAs share a
 // head and each moves a quarter of W^UK_h; the weight quarter lands as two TMA boxes
 // ([128 x 64] chunks, 128-byte swizzle) and is the MN-major A operand (M = latent
-// column, K = head dim) of 8 MMAs against the staged q_nope rows (N = rows).
-// merge: one CTA per (32 latent columns, sequence, row group), four threads per row sharing the
-// sequence's pieces (the attend kernel writes them in [column group][row] order)
-// and writes o_lat into per-(head, 64-row block) tiles already in the swizzled K-major
-// operand layout, so the up-projection takes its operand with one bulk copy.
-// upproj: one CTA per (head, up to 64 rows); W^UV_h (eight [128 x 64] TMA boxes) is
-// requested before the CTA waits for the merge, so the weight load overlaps it.
+// column, K = head dim) of 8 MMAs against the staged q_nope rows (N = rows).  (One CTA per
+// head with all four quarters measured slower: 15.1 against 13.6 us at T = 32, 68.9 against
+// 35.9 us at T = 256, ncu.)
+// merge: one CTA per (32 latent columns, sequence, row group), 1, 2 or 4 threads per row sharing
+// the sequence's pieces (the attend kernel writes them in [column group][row] order); it writes
+// o_lat into per-(head, 256-row block) tiles already in the swizzled K-major operand layout, so
+// each K step of the up-projection takes its operand with one bulk copy.
+// upproj: one CTA per (head, up to 256 rows), the contraction over the latent columns streamed
+// through a four-stage ring; W^UV_h's first chunks are requested before the CTA waits for the
+// merge, so the weight load overlaps it.
+// upproj stages its bf16 result in shared memory and writes whole output rows with 16-byte stores.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -33,9 +37,9 @@ using namespace sm100;
 
 namespace proj {
 
-constexpr int kTokBlock = 64;                // query rows per CTA
 constexpr int kWChunkBytes = 128 * 64 * 2;   // [128 rows x 64 columns] bf16 = 16 KB
 constexpr int kWBytes = 8 * kWChunkBytes;    // one head's weight matrix, 128 KB
+constexpr int kTokBlock = 64;                // absorb: query rows per CTA
 constexpr uint64_t kLimitNs = 2000000000ull;
 
 // 16-byte unit u (0..7) of row r in a 128-byte swizzled row of a [rows x 64] chunk
@@ -205,13 +209,15 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
 constexpr int kMergeSlices = 16;    // a CTA merges 32 of the 512 latent columns (8 column groups of 4)
 
 // Byte offset of row t of head h, latent unit (chunk c, unit u) in the o_lat tiles: per head, the rows
-// are cut into blocks of 64 (the last one olat_rows(T) - 64 * (blocks - 1) rows); a block is eight
-// [rows x 64] chunks, each 128-byte swizzled, so it is the K-major B operand of the up-projection.
+// are cut into blocks of kOlatBlock (the last one olat_rows(T) - kOlatBlock * (blocks - 1) rows); a block
+// is eight [rows x 64] chunks, each 128-byte swizzled, so chunk c of a block is the K-major B operand of
+// the up-projection's K step c and arrives with one bulk copy.
+constexpr int kOlatBlock = 256;
 __device__ __forceinline__ int64_t olat_offset(int T, int h, int t, int c, int u) {
     const int Tp = olat_rows(T);
-    const int tb = t >> 6, i = t & 63;
-    const int rows = min(64, Tp - 64 * tb);
-    return (static_cast<int64_t>(h) * Tp + 64 * tb) * 1024 + c * rows * 128 + swz(i, u);
+    const int tb = t / kOlatBlock, i = t % kOlatBlock;
+    const int rows = min(kOlatBlock, Tp - kOlatBlock * tb);
+    return (static_cast<int64_t>(h) * Tp + kOlatBlock * tb) * 1024 + c * rows * 128 + swz(i, u);
 }
 
 // One CTA per (32-column slice, sequence, row group).  Row r of the group is merged by kSplit threads
@@ -337,80 +343,99 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
 // ------------------------------------------------------------------ up-projection
 
 constexpr int kUpThreads = 128;
-constexpr int kUpOffW = 0;
-constexpr int kUpOffB = kWBytes;                      // o_lat tile, up to 64 rows x 1 KB
-constexpr int kUpOffBar = kUpOffB + kTokBlock * 1024;
-constexpr int kUpSmemBytes = kUpOffBar + 64;
+constexpr int kUpRows = kOlatBlock;                        // o_lat rows per CTA = one o_lat block (MMA N <= 256)
+constexpr int kUpStages = 4;                               // ring of K chunks (8 per head)
+constexpr int kUpOffB = kWChunkBytes;                      // stage: W^UV chunk (16 KB) | o_lat chunk (<= 32 KB)
+constexpr int kUpStageBytes = kWChunkBytes + kUpRows * 128;
+constexpr int kUpOffBar = kUpStages * kUpStageBytes;
+constexpr int kUpSmemBytes = kUpOffBar + 128;
+static_assert(kUpStageBytes % 1024 == 0 && kUpRows * kDh * 2 <= kUpOffBar, "stages 1024-aligned; output staging fits");
 
-// One head's weights as eight [128 x 64] boxes (one per 64-column chunk): several boxes in flight
-// stream far faster through the TMA unit than one 128 KB box.
-__device__ __forceinline__ void tma_load_w(uint32_t dst, const CUtensorMap* map, int head, uint64_t* bar) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) tma_load_3d(dst + c * kWChunkBytes, map, 0, head * 128, c, bar);
-}
-
+// One CTA per (head, block of up to 256 o_lat rows).  The contraction over the 512 latent columns streams
+// through a ring of four stages, one 64-column chunk per stage: W^UV_h's chunk as a [128 x 64] TMA box (the
+// K-major A operand, M = output dim) and the o_lat block's chunk as one bulk copy (the K-major B operand,
+// N = rows).  W^UV is an input of the decode call, never written by the kernels before this one in it, so
+// its first boxes are requested before the CTA waits for the merge.  The result is staged in shared memory
+// as bf16 rows and leaves as 16-byte stores (each output row is 256 contiguous bytes).
 __global__ void __launch_bounds__(kUpThreads) upproj_kernel(const __grid_constant__ CUtensorMap wuv_map,
                                                            const uint8_t* __restrict__ olat, int T, int H,
                                                            uint16_t* __restrict__ out, int32_t* dev_status) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kUpOffBar);  // 0: weights, 1: o_lat, 2: MMA done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kUpOffBar + 32);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kUpOffBar);  // full[4], empty[4], done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kUpOffBar + 8 * (2 * kUpStages + 1));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x;
-    const int t0 = blockIdx.y * kTokBlock;
-    const int nt = min(kTokBlock, T - t0);
+    const int t0 = blockIdx.y * kUpRows;
+    const int nt = min(kUpRows, T - t0);
     const int Tp = olat_rows(T);
-    const int NT = min(kTokBlock, Tp - t0);  // rows of this o_lat tile (a multiple of 16)
+    const int NT = min(kUpRows, Tp - t0);  // rows of this o_lat block (a multiple of 16)
+    const uint32_t chunk_bytes = static_cast<uint32_t>(NT) * 128u;
+    const uint8_t* blk = olat + (static_cast<int64_t>(h) * Tp + t0) * 1024;  // chunk c at c * NT * 128
     volatile int never = 0;
     if ((sbase & 1023u) != 0) {
         if (tid == 0) report(dev_status, MLA_DEVERR_TIMEOUT);
         return;
     }
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 2 * kUpStages + 1; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         prefetch_tmap(&wuv_map);
-        // W^UV is an input of the decode call, never written by the kernels before this one in it
-        mbar_arrive_expect_tx(&bars[0], kWBytes);
-        tma_load_w(sbase + kUpOffW, &wuv_map, h, &bars[0]);
+        for (int c = 0; c < kUpStages; ++c) {
+            mbar_arrive_expect_tx(&bars[c], kWChunkBytes + chunk_bytes);
+            tma_load_3d(sbase + c * kUpStageBytes, &wuv_map, 0, h * 128, c, &bars[c]);
+        }
     }
-    if (warp == 0) tmem_alloc(tmem_slot, 64);
+    if (warp == 0) tmem_alloc(tmem_slot, 256);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     grid_dependency_wait();  // o_lat comes from the merge kernel
     bool ok = true;
-    if (tid == 0) {
-        const uint32_t bytes = static_cast<uint32_t>(NT) * 1024u;
-        mbar_arrive_expect_tx(&bars[1], bytes);
-        bulk_load_hint(sbase + kUpOffB, olat + (static_cast<int64_t>(h) * Tp + t0) * 1024, bytes, &bars[1],
-                       l2_policy_evict_first());
-        ok = mbar_wait(&bars[0], 0, &never, kLimitNs) && mbar_wait(&bars[1], 0, &never, kLimitNs);
-        if (ok) {
-            tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(128, NT, false, false);
-            const uint64_t a0 = sdesc_sw128(sbase + kUpOffW, 16, 1024);
-            const uint64_t b0 = sdesc_sw128(sbase + kUpOffB, 16, 1024);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const uint64_t ad = a0 + static_cast<uint64_t>(((k >> 2) * kWChunkBytes + (k & 3) * 32) >> 4);
-                const uint64_t bd = b0 + static_cast<uint64_t>(((k >> 2) * NT * 128 + (k & 3) * 32) >> 4);
-                mma_ss(tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
-            }
-            mma_commit(smem_u32(&bars[2]));
-        } else {
-            report(dev_status, MLA_DEVERR_TIMEOUT);
+    if (warp == 0 && lane == 0) {
+        // producer: the o_lat halves of the first four stages, then both halves of chunks 4..7 as stages free
+        const uint64_t once = l2_policy_evict_first();
+        for (int c = 0; c < kUpStages; ++c)
+            bulk_load_hint(sbase + c * kUpStageBytes + kUpOffB, blk + c * chunk_bytes, chunk_bytes, &bars[c], once);
+        for (int c = kUpStages; ok && c < 8; ++c) {
+            const int s = c % kUpStages;
+            ok = mbar_wait(&bars[kUpStages + s], 0, &never, kLimitNs);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&bars[s], kWChunkBytes + chunk_bytes);
+            tma_load_3d(sbase + s * kUpStageBytes, &wuv_map, 0, h * 128, c, &bars[s]);
+            bulk_load_hint(sbase + s * kUpStageBytes + kUpOffB, blk + c * chunk_bytes, chunk_bytes, &bars[s], once);
         }
+        if (!ok) report(dev_status, MLA_DEVERR_TIMEOUT);
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer: out^T[d, t] += W^UV_h[d, chunk] o_lat[t, chunk], four K = 16 steps per chunk
+        const uint32_t idesc = idesc_bf16_f32(128, NT, false, false);
+        for (int c = 0; ok && c < 8; ++c) {
+            const int s = c % kUpStages;
+            ok = mbar_wait(&bars[s], static_cast<uint32_t>(c / kUpStages), &never, kLimitNs);
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t a0 = sdesc_sw128(sbase + s * kUpStageBytes, 16, 1024);
+            const uint64_t b0 = sdesc_sw128(sbase + s * kUpStageBytes + kUpOffB, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tmem, a0 + static_cast<uint64_t>((kk * 32) >> 4), b0 + static_cast<uint64_t>((kk * 32) >> 4),
+                       idesc, (c > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(smem_u32(&bars[kUpStages + s]));  // stage s free once these MMAs are done
+        }
+        if (!ok) report(dev_status, MLA_DEVERR_TIMEOUT);
+        mma_commit(smem_u32(&bars[2 * kUpStages]));  // also after a failure: TMEM is freed only once it fires
     }
     ok = __syncthreads_and(ok);
-    if (ok) {
-        const bool done = mbar_wait(&bars[2], 0, &never, kLimitNs);
+    {
+        const bool done = mbar_wait(&bars[2 * kUpStages], 0, &never, kLimitNs);
         __syncwarp();
         tc_fence_after();
-        if (__all_sync(0xffffffffu, done)) {
-            const int d = 32 * warp + lane;  // output row of W^UV_h
+        ok = __all_sync(0xffffffffu, done) && ok;
+        if (ok) {
+            // D: lane d = output dim of W^UV_h, column j = row t0 + j.  Every MMA is done, so the stages are
+            // free: row j of the result goes to [j * 256, j * 256 + 256) as bf16
+            const int d = 32 * warp + lane;
             for (int j0 = 0; j0 < NT; j0 += 32) {
                 uint32_t v[32];
                 const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + j0;
@@ -421,17 +446,26 @@ __global__ void __launch_bounds__(kUpThreads) upproj_kernel(const __grid_constan
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
                     if (j < jn)
-                        out[(static_cast<int64_t>(t0 + j0 + j) * H + h) * kDh + d] = f32_to_bf16_rne(__uint_as_float(v[j]));
+                        *reinterpret_cast<uint16_t*>(smem + (j0 + j) * (kDh * 2) + 2 * d) =
+                            f32_to_bf16_rne(__uint_as_float(v[j]));
             }
-        } else if (lane == 0) {
+        } else if (lane == 0 && !done) {
             report(dev_status, MLA_DEVERR_TIMEOUT);
+        }
+    }
+    ok = __syncthreads_and(ok);
+    if (ok) {
+        for (int i = tid; i < nt * (kDh * 2 / 16); i += kUpThreads) {
+            const int j = i / (kDh * 2 / 16), q = i % (kDh * 2 / 16);
+            reinterpret_cast<uint4*>(out + (static_cast<int64_t>(t0 + j) * H + h) * kDh)[q] =
+                *reinterpret_cast<const uint4*>(smem + j * (kDh * 2) + 16 * q);
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 64);
+        tmem_dealloc(tmem, 256);
     }
 }
 
@@ -518,7 +552,7 @@ cudaError_t launch_upproj(const uint8_t* olat, const uint16_t* W_UV, int T, int 
     cudaError_t e = cudaFuncSetAttribute(proj::upproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          proj::kUpSmemBytes);
     if (e != cudaSuccess) return e;
-    const dim3 grid(H, (T + proj::kTokBlock - 1) / proj::kTokBlock);
+    const dim3 grid(H, (T + proj::kUpRows - 1) / proj::kUpRows);
     return proj::launch_pdl(proj::upproj_kernel, grid, proj::kUpThreads, proj::kUpSmemBytes, stream, map, olat, T, H,
                             out, dev_status);
 }
