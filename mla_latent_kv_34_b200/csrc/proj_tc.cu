@@ -11,7 +11,7 @@
 //  upproj:  out[t, h, :] = W^UV_h o_lat[t, h, :]                   (128 = 128 x 512)
 //           W^UV is applied after the aggregation in latent space ("两张账" page).
 //
-// absorb: one CTA per (128 latent columns, head, up to 64 query rows), so 4 CTAs share a
+// absorb: one CTA per (128 latent columns, head, up to 128 query rows), so 4 CTAs share a
 // head and each moves a quarter of W^UK_h; the weight quarter lands as two TMA boxes
 // ([128 x 64] chunks, 128-byte swizzle) and is the MN-major A operand (M = latent
 // column, K = head dim) of 8 MMAs against the staged q_nope rows (N = rows).  (One CTA per
@@ -39,7 +39,7 @@ namespace proj {
 
 constexpr int kWChunkBytes = 128 * 64 * 2;   // [128 rows x 64 columns] bf16 = 16 KB
 constexpr int kWBytes = 8 * kWChunkBytes;    // one head's weight matrix, 128 KB
-constexpr int kTokBlock = 64;                // absorb: query rows per CTA
+constexpr int kTokBlock = 128;               // absorb: query rows per CTA (MMA N <= 128)
 constexpr uint64_t kLimitNs = 2000000000ull;
 
 // 16-byte unit u (0..7) of row r in a 128-byte swizzled row of a [rows x 64] chunk
@@ -49,8 +49,9 @@ __device__ __forceinline__ uint32_t swz(int r, int u) { return static_cast<uint3
 
 constexpr int kAbsThreads = 128;
 constexpr int kAbsOffW = 0;                              // two weight chunks, 32 KB
-constexpr int kAbsOffB = 2 * kWChunkBytes;               // q_nope rows: two [NT x 64] chunks, <= 16 KB
-constexpr int kAbsOffBar = kAbsOffB + kTokBlock * 128 * 2;
+constexpr int kAbsOffB = 2 * kWChunkBytes;               // q_nope rows: two [NT x 64] chunks, <= 32 KB
+constexpr int kAbsOffPos = kAbsOffB + kTokBlock * 128 * 2;  // query positions of the rows (RoPE CTAs)
+constexpr int kAbsOffBar = kAbsOffPos + kTokBlock * 4;
 constexpr int kAbsSmemBytes = kAbsOffBar + 64;
 
 __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
@@ -78,30 +79,44 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
         fence_mbar_init();
         prefetch_tmap(&wuk_map);
     }
-    if (warp == 0) tmem_alloc(tmem_slot, 64);
+    if (warp == 0) tmem_alloc(tmem_slot, kTokBlock);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    int32_t* pos_s = reinterpret_cast<int32_t*>(smem + kAbsOffPos);
     grid_dependency_wait();  // inputs may come from the previous kernel on the stream
+    // query positions of the RoPE CTAs' rows (-1: none given; -2: outside the table, reported, and that
+    // row's RoPE part is left unwritten)
+    if (mb == 0 && tid < nt) {
+        int32_t pp = -1;
+        if (pos) {
+            pp = pos[t0 + tid];
+            if (pp < 0 || pp >= rope_len) {
+                report(dev_status, MLA_DEVERR_POS_RANGE);
+                pp = -2;
+            }
+        }
+        pos_s[tid] = pp;
+    }
     if (tid == 0) {
         mbar_arrive_expect_tx(&bars[0], 2 * kWChunkBytes);
         tma_load_3d(sbase + kAbsOffW, &wuk_map, 0, h * 128, 2 * mb, &bars[0]);
         tma_load_3d(sbase + kAbsOffW + kWChunkBytes, &wuk_map, 0, h * 128, 2 * mb + 1, &bars[0]);
     }
-    // B operand: q_nope rows t (N) x 128 (K), two swizzled [NT x 64] chunks; rows >= nt are zero.
-    {
-        constexpr int kIt = kTokBlock * 16 / kAbsThreads;
-        uint4 v[kIt];
+    // B operand: q_nope rows t (N) x 128 (K), two swizzled [NT x 64] chunks; rows >= nt are zero.  Eight
+    // 16-byte loads per thread in flight at a time.
+    for (int base = 0; base < NT * 16; base += 8 * kAbsThreads) {
+        uint4 v[8];
 #pragma unroll
-        for (int k = 0; k < kIt; ++k) {
-            const int idx = tid + k * kAbsThreads, r = idx >> 4, u16 = idx & 15;  // 16 units of 16 B per row
+        for (int k = 0; k < 8; ++k) {
+            const int idx = base + tid + k * kAbsThreads, r = idx >> 4, u16 = idx & 15;  // 16 units per row
             v[k] = make_uint4(0, 0, 0, 0);
             if (r < nt) v[k] = reinterpret_cast<const uint4*>(q_nope + (static_cast<int64_t>(t0 + r) * H + h) * kDh)[u16];
         }
 #pragma unroll
-        for (int k = 0; k < kIt; ++k) {
-            const int idx = tid + k * kAbsThreads, r = idx >> 4, u16 = idx & 15;
+        for (int k = 0; k < 8; ++k) {
+            const int idx = base + tid + k * kAbsThreads, r = idx >> 4, u16 = idx & 15;
             if (r < NT) *reinterpret_cast<uint4*>(smem + kAbsOffB + (u16 >> 3) * NT * 128 + swz(r, u16 & 7)) = v[k];
         }
     }
@@ -128,47 +143,50 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
         }
     }
     grid_dependents_launch();
-    // RoPE part on CUDA cores meanwhile (one CTA per head and row block does it): nt rows x 32 pairs,
-    // the same arithmetic as the cache append.  Thread tid owns pair tid % 32 of rows tid / 32 + 4 k.
+    // RoPE part on CUDA cores meanwhile (the first CTA of each head and row block does it), the same
+    // arithmetic as the cache append.  A thread takes 16-byte units (row j, dims 8u .. 8u + 7 = pairs
+    // 4u .. 4u + 3) four at a time, with every load of a batch in flight together; the positions were
+    // staged before the first barrier above.
     if (mb == 0) {
-        constexpr int kIt = kTokBlock * (kDr / 2) / kAbsThreads;
-        const int pr = tid & 31;
-        uint32_t xr[kIt];
-        int32_t pp[kIt];
+        for (int base = 0; base < nt * 8; base += 4 * kAbsThreads) {
+            uint4 x[4];
+            float4 cs[4][2];
 #pragma unroll
-        for (int k = 0; k < kIt; ++k) {
-            const int t = (tid >> 5) + k * (kAbsThreads / 32);
-            xr[k] = 0u;
-            pp[k] = 0;
-            if (t < nt) {
-                xr[k] = reinterpret_cast<const uint32_t*>(q_rope + (static_cast<int64_t>(t0 + t) * H + h) * kDr)[pr];
-                if (pos) pp[k] = pos[t0 + t];
-            }
-        }
-        float2 cs[kIt];
-#pragma unroll
-        for (int k = 0; k < kIt; ++k) {
-            const int t = (tid >> 5) + k * (kAbsThreads / 32);
-            cs[k] = make_float2(1.f, 0.f);
-            if (t < nt && pos && pp[k] >= 0 && pp[k] < rope_len)
-                cs[k] = reinterpret_cast<const float2*>(rope_table + static_cast<int64_t>(pp[k]) * kDr)[pr];
-        }
-#pragma unroll
-        for (int k = 0; k < kIt; ++k) {
-            const int t = (tid >> 5) + k * (kAbsThreads / 32);
-            if (t >= nt) continue;
-            uint32_t y = xr[k];
-            if (pos) {
-                if (pp[k] < 0 || pp[k] >= rope_len) {
-                    report(dev_status, MLA_DEVERR_POS_RANGE);
-                    continue;
+            for (int k = 0; k < 4; ++k) {
+                const int idx = base + tid + k * kAbsThreads, j = idx >> 3, u = idx & 7;
+                x[k] = make_uint4(0, 0, 0, 0);
+                cs[k][0] = cs[k][1] = make_float4(1.f, 0.f, 1.f, 0.f);
+                if (j < nt) {
+                    x[k] = reinterpret_cast<const uint4*>(q_rope + (static_cast<int64_t>(t0 + j) * H + h) * kDr)[u];
+                    const int32_t pp = pos_s[j];
+                    if (pp >= 0) {
+                        const float4* row = reinterpret_cast<const float4*>(rope_table + static_cast<int64_t>(pp) * kDr);
+                        cs[k][0] = row[2 * u];
+                        cs[k][1] = row[2 * u + 1];
+                    }
                 }
-                const float x0 = bf16_to_f32(static_cast<uint16_t>(xr[k] & 0xFFFFu));
-                const float x1 = bf16_to_f32(static_cast<uint16_t>(xr[k] >> 16));
-                y = pack_bf16x2(__fsub_rn(__fmul_rn(x0, cs[k].x), __fmul_rn(x1, cs[k].y)),
-                                __fadd_rn(__fmul_rn(x0, cs[k].y), __fmul_rn(x1, cs[k].x)));
             }
-            reinterpret_cast<uint32_t*>(q_out + (static_cast<int64_t>(t0 + t) * H + h) * kRow + kDc)[pr] = y;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int idx = base + tid + k * kAbsThreads, j = idx >> 3, u = idx & 7;
+                if (j >= nt || pos_s[j] == -2) continue;
+                uint4 y = x[k];
+                if (pos_s[j] >= 0) {
+                    const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+                    const float c[8] = {cs[k][0].x, cs[k][0].y, cs[k][0].z, cs[k][0].w,
+                                        cs[k][1].x, cs[k][1].y, cs[k][1].z, cs[k][1].w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {  // pair 4u + e: (cos, sin) = (c[2e], c[2e + 1])
+                        const float x0 = bf16_to_f32(static_cast<uint16_t>(w[e] & 0xFFFFu));
+                        const float x1 = bf16_to_f32(static_cast<uint16_t>(w[e] >> 16));
+                        o[e] = pack_bf16x2(__fsub_rn(__fmul_rn(x0, c[2 * e]), __fmul_rn(x1, c[2 * e + 1])),
+                                           __fadd_rn(__fmul_rn(x0, c[2 * e + 1]), __fmul_rn(x1, c[2 * e])));
+                    }
+                    y = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(t0 + j) * H + h) * kRow + kDc)[u] = y;
+            }
         }
     }
     ok = __syncthreads_and(ok);
@@ -200,7 +218,7 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 64);
+        tmem_dealloc(tmem, kTokBlock);
     }
 }
 

@@ -205,10 +205,12 @@ def test_decode_multi_token_queries(cuda_ok, H, n_q, Hh, L):
     _check_decode(prob, out, lse, [0, 1, 2], label=f"n_q={n_q}")
 
 
-@pytest.mark.parametrize("n_q,Hh,L", [(32, 16, 600), (100, 8, 400), (256, 16, 700), (64, 128, 300)])
+@pytest.mark.parametrize("n_q,Hh,L", [(32, 16, 600), (100, 8, 400), (256, 16, 700), (64, 128, 300),
+                                      (150, 4, 500)])
 def test_decode_prefill_chunks(cuda_ok, H, n_q, Hh, L):
     """Chunks of up to 256 new tokens per sequence in the absorbed form (the arithmetic favours it
-    over the naive form below about 340 tokens); query j sees keys up to L - n_q + j."""
+    over the naive form below about 340 tokens); query j sees keys up to L - n_q + j.  T = 2 n_q query
+    rows: 300 rows span two 256-row blocks of the merged latent output, the second a partial one."""
     cfg = mi.MLAConfig("chunk", B=2, H=Hh, n_q=n_q, L=L, seed=3000 + n_q + Hh)
     prob = H.build_problem(cfg, lengths=[L, max(n_q, L // 2)], shuffle_seed=n_q)
     q = prob.absorb()
