@@ -36,6 +36,9 @@ mla_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_E
 
 int max_pairs_per_group(int G) { return kMaxPairs / G > 1 ? kMaxPairs / G : 1; }
 
+// Few query rows (n_q * H <= 32): the one-SM kernel (one row group, up to kMaxSmCtas CTAs) instead of CTA pairs.
+bool one_sm_path(int n_q, int H) { return static_cast<int64_t>(n_q) * H <= kMaxSmRows; }
+
 // ---- tensor-core path: segment partials [G][slots][128 rows] float2 (m, l), then (1024-aligned)
 //      [G][slots] blocks of 128 rows x 512 fp32 O, each stored as [128 column groups of 4][128 rows] x float4,
 //      then (1024-aligned) the merged latent output o_lat as bf16 operand tiles, [H][olat_rows(T)] x 1 KB.
@@ -50,8 +53,9 @@ size_t align1k(size_t x) { return ((x + 1023) / 1024) * 1024; }
 TcWs tc_ws_layout(int B, int n_q, int H) {
     TcWs w;
     w.G = (n_q * H + 127) / 128;
-    // a group gets at most max(1, kMaxPairs / G) CTA pairs (long query chunks: many groups, few pairs each)
-    w.slots = B + max_pairs_per_group(w.G);
+    // a group gets at most max(1, kMaxPairs / G) CTA pairs (long query chunks: many groups, few pairs each);
+    // with few query rows the one-SM kernel's up to kMaxSmCtas CTAs share the single group
+    w.slots = B + (one_sm_path(n_q, H) ? kMaxSmCtas : max_pairs_per_group(w.G));
     const size_t rows = static_cast<size_t>(w.G) * w.slots * 128;
     w.ml_part = 0;
     w.o_part = align1k(rows * sizeof(float2));
@@ -60,7 +64,15 @@ TcWs tc_ws_layout(int B, int n_q, int H) {
     return w;
 }
 
-int tc_clusters_per_group(int G, int num_splits) {
+// Work units (CTA pairs, or CTAs of the one-SM kernel) per row group; the attend and finish phases derive
+// the same number, so the merge finds every piece.
+int tc_clusters_per_group(int G, int num_splits, bool one_sm) {
+    if (one_sm) {
+        int n = decode_sm_ctas();
+        if (n <= 0) return 0;
+        if (num_splits > 0 && num_splits < n) n = num_splits;
+        return n;
+    }
     const int total = decode_tc_clusters();
     if (total <= 0) return 0;
     int pg = total / G;
@@ -200,9 +212,16 @@ mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_block
     if (!aligned16(q) || !aligned16(cache) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
     const TcWs lay = tc_ws_layout(B, n_q, H);
     if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
-    const int pg = tc_clusters_per_group(lay.G, num_splits);
+    const bool one_sm = one_sm_path(n_q, H);
+    const int pg = tc_clusters_per_group(lay.G, num_splits, one_sm);
     if (pg <= 0) return MLA_ERR_CUDA;
     char* ws = static_cast<char*>(workspace);
+    if (one_sm)
+        return cuda_status(launch_decode_sm(static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(cache),
+                                            cap_blocks, block_table, max_blocks, kv_len, B, n_q, H, scale, pg,
+                                            reinterpret_cast<float*>(ws + lay.o_part),
+                                            reinterpret_cast<float2*>(ws + lay.ml_part), lay.slots, dev_status,
+                                            static_cast<cudaStream_t>(stream)));
     return cuda_status(launch_decode_tc(static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(cache),
                                         cap_blocks, block_table, max_blocks, kv_len, B, n_q, H, scale, pg,
                                         reinterpret_cast<float*>(ws + lay.o_part),
@@ -220,7 +239,7 @@ mla_status mla_decode_finish(const int32_t* kv_len, int max_blocks, const void* 
     if (!aligned16(W_UV) || !aligned16(out) || !aligned16(workspace)) return MLA_ERR_INVALID_ARG;
     const TcWs lay = tc_ws_layout(B, n_q, H);
     if (ws_bytes < lay.total) return MLA_ERR_WORKSPACE;
-    const int pg = tc_clusters_per_group(lay.G, num_splits);
+    const int pg = tc_clusters_per_group(lay.G, num_splits, one_sm_path(n_q, H));
     if (pg <= 0) return MLA_ERR_CUDA;
     char* ws = static_cast<char*>(workspace);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);

@@ -20,6 +20,8 @@ constexpr int kBlockBytes = MLA_BLOCK_BYTES;    // 9 chunks x [128 rows x 128 B]
 constexpr int kBlockChunk = kBlockTokens * 128;  // bytes of one 64-column chunk of a block
 static_assert(kBlockBytes == 9 * kBlockChunk, "block layout");
 constexpr int kMaxPairs = 74;      // CTA pairs per row group the tensor-core decode uses at most (148 SMs / 2)
+constexpr int kMaxSmRows = 32;     // query rows (n_q * H) up to which the one-SM decode kernel runs instead
+constexpr int kMaxSmCtas = 148;    // CTAs the one-SM decode kernel uses at most (one per SM)
 
 // Tiles (128-token blocks) of a sequence that the decode processes: none when kv_len < n_q or when the
 // sequence needs more blocks than its block-table row holds.  The attend and merge kernels both use this
@@ -92,6 +94,10 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int T, in
 
 // Tensor-core decode (decode_tc.cu); the merge of its pieces and the W^UV projection (proj_tc.cu).
 int decode_tc_clusters();
+int decode_sm_ctas();
+cudaError_t launch_decode_sm(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
+                             int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale, int ctas,
+                             float* o_part, float2* ml_part, int slots, int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
                              int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale,
                              int clusters_per_group, float* o_part, float2* ml_part, int slots, int32_t* dev_status,

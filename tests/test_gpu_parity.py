@@ -250,6 +250,28 @@ def test_decode_split_invariance(cuda_ok, H, splits):
     _check_decode(prob, out, lse, [0, 2], label=f"splits={splits}")
 
 
+@pytest.mark.parametrize("B,Hh,n_q,L_max,splits,shuffle", [(7, 16, 2, 1500, 0, 3), (3, 4, 1, 700, 0, None),
+                                                          (5, 11, 2, 2000, 3, 5), (1, 1, 1, 5, 0, None),
+                                                          (40, 16, 1, 600, 1, 7), (6, 32, 1, 2600, 0, 9),
+                                                          (4, 16, 2, 300, 200, None)])
+def test_decode_few_rows_one_sm_kernel(cuda_ok, H, B, Hh, n_q, L_max, splits, shuffle):
+    """At most 32 query rows (n_q * H): the one-SM kernel (tokens as the MMA's M side, both contractions on
+    one SM), with shuffled block tables and NaN canaries in unowned blocks, against the CUDA-core path and
+    the oracle; one work unit per SM down to a single one, and more units than tiles."""
+    cfg = mi.MLAConfig("one-sm", B=B, H=Hh, n_q=n_q, L=None, L_max=L_max, seed=700 + B + Hh + n_q)
+    prob = H.build_problem(cfg, shuffle_seed=shuffle)
+    q = prob.absorb()
+    ref_out, ref_lse = prob.decode(q, num_splits=3, path="cudacore")
+    out, lse = prob.decode(q, num_splits=splits)
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    assert torch.isfinite(out.float()).all()
+    a, b = out.float().cpu().numpy(), ref_out.float().cpu().numpy()
+    assert np.all(np.abs(a - b) <= 2 * (ATOL + RTOL * np.abs(b)))
+    assert np.abs(lse.cpu().numpy() - ref_lse.cpu().numpy()).max() < 2e-2
+    _check_decode(prob, out, lse, range(min(B, 6)), label=f"one-sm B={B} H={Hh} n_q={n_q}")
+
+
 def test_decode_ignores_rows_outside_sequences(cuda_ok, H):
     """NaN rows between and after sequences never leak into any result."""
     cfg = mi.MLAConfig("gaps", B=5, H=128, n_q=2, L=None, L_max=400, seed=66)
