@@ -16,8 +16,8 @@
 // and one SM does the whole tile: each cache block is read from HBM once, by one SM, and nothing crosses
 // SMs.  NR = 16 or 32 (the rows rounded up).
 //
-// Softmax: a thread per token (tensor-memory lane).  Row maxima by warp shuffles and an exchange of the
-// four warps' maxima through shared memory; the running maximum is stale (it moves only when a tile's
+// Softmax: a thread per token (tensor-memory lane).  Row maxima by a warp reduction and an exchange of
+// the four warps' maxima through shared memory; the running maximum is stale (it moves only when a tile's
 // maximum exceeds it by more than 2^8, and then O^T is rescaled in tensor memory); each thread keeps its
 // token lane's share of every row sum, and the shares are added once per segment.  P goes to shared
 // memory as bf16 in the swizzled K-major layout of the second MMA's B operand.
@@ -142,6 +142,13 @@ struct SegWalk {
 __device__ __forceinline__ void raise_abort(volatile int* abort_flag, int32_t* dev_status) {
     *abort_flag = 1;
     if (dev_status) atomicOr(dev_status, MLA_DEVERR_TIMEOUT);
+}
+
+// Maximum over the warp's 32 lanes (sm_100a warp reduction; inputs are finite or -inf).
+__device__ __forceinline__ float warp_max_f32(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
 }
 
 template <int NR>
@@ -287,14 +294,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm_kernel(const Params p) 
             for (int t = s.t0; ok && t < s.t1; ++t, ++n) {
                 const uint32_t sb = n & 1u, us = n >> 1;
                 const bool first = (t == s.t0);
+                const int nvalid = min(kTile, s.L - t * kTile);
                 if (lane == 0) {
                     ok = mbar_wait(&bars[kBSEmpty + sb], (us & 1u) ^ 1u, abort_flag, kLimitNs);
-                    for (int k = 0; ok && k < kSlots; ++k)
+                    // a partial block waits for all three copies (its V rows past the end are zeroed first);
+                    // a full one starts each copy's 12 MMAs as soon as that copy has landed
+                    for (int k = 0; ok && nvalid < kTile && k < kSlots; ++k)
                         ok = mbar_wait(&bars[kBFull + k], n & 1u, abort_flag, kLimitNs);
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
-                const int nvalid = min(kTile, s.L - t * kTile);
                 if (nvalid < kTile) {
                     // rows past the sequence end: P is 0 there, make V 0 too (no 0 * NaN); their scores are masked
                     const int nz = (kTile - nvalid) * 8;  // 16-byte units per chunk
@@ -307,20 +316,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm_kernel(const Params p) 
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    tc_fence_after();
                     // S^T = K Q^T into score buffer sb
                     const uint32_t d = tmem + L::col_s(sb);
+                    for (int k = 0; ok && k < kSlots; ++k) {
+                        if (nvalid == kTile) ok = mbar_wait(&bars[kBFull + k], n & 1u, abort_flag, kLimitNs);
+                        if (!ok) break;
+                        tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < 9; ++c)
+                        for (int j = 0; j < 3; ++j)
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(d, ring_desc + static_cast<uint64_t>((c * kChunk + kk * 32) >> 4),
-                                   q_desc + static_cast<uint64_t>((c * L::kQChunk + kk * 32) >> 4), idesc_s,
-                                   (c | kk) ? 1u : 0u);
-                    mma_commit(smem_u32(&bars[kBSFull + sb]));
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const int c = 3 * k + j;
+                                mma_ss(d, ring_desc + static_cast<uint64_t>((c * kChunk + kk * 32) >> 4),
+                                       q_desc + static_cast<uint64_t>((c * L::kQChunk + kk * 32) >> 4), idesc_s,
+                                       (c | kk) ? 1u : 0u);
+                            }
+                    }
+                    if (ok) mma_commit(smem_u32(&bars[kBSFull + sb]));
                     // O^T += V^T P^T once the softmax has staged P (and, at a segment's first tile, the
                     // epilogue has read the previous segment's O^T)
-                    ok = mbar_wait(&bars[kBPReady + sb], us & 1u, abort_flag, kLimitNs);
+                    ok = ok && mbar_wait(&bars[kBPReady + sb], us & 1u, abort_flag, kLimitNs);
                     if (ok && first) ok = mbar_wait(&bars[kBOFree], (kseg & 1u) ^ 1u, abort_flag, kLimitNs);
                     if (ok) {
                         tc_fence_after();
@@ -389,15 +404,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm_kernel(const Params p) 
             fence_proxy_async_cta();
             tc_fence_before();
             mbar_arrive(&bars[kBQReady]);
-            // visible keys of row r: 0 .. L - n_q + r / H
+            // visible keys of row r (query j = r / H): 0 .. L - n_q + j
             float m[NR], lp[NR];
-            int lim[NR];
 #pragma unroll
             for (int r = 0; r < NR; ++r) {
                 m[r] = -CUDART_INF_F;
                 lp[r] = 0.f;
-                lim[r] = r < p.R ? s.L - p.n_q + r / p.H + 1 : 0;
             }
+            const int lim0 = s.L - p.n_q + 1;  // keys below this are visible to every query of the step
             for (int t = s.t0; t < s.t1; ++t, ++n) {
                 const uint32_t sb = n & 1u, us = n >> 1;
                 bool ok = mbar_wait(&bars[kBSFull + sb], us & 1u, abort_flag, kLimitNs);
@@ -408,15 +422,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm_kernel(const Params p) 
                 tc_fence_before();
                 mbar_arrive(&bars[kBSEmpty + sb]);
                 const int tok = t * kTile + tk;
+                if (tok < lim0) {
 #pragma unroll
-                for (int r = 0; r < NR; ++r) sv[r] = tok < lim[r] ? sv[r] : -CUDART_INF_F;
+                    for (int r = 0; r < NR; ++r) sv[r] = r < p.R ? sv[r] : -CUDART_INF_F;
+                } else {
+#pragma unroll
+                    for (int r = 0; r < NR; ++r) sv[r] = (r < p.R && tok < lim0 + r / p.H) ? sv[r] : -CUDART_INF_F;
+                }
                 // row maxima over the tile's 128 tokens: warp shuffles, then the four warps' maxima
                 float* rmax = red + sb * 4 * NR;
 #pragma unroll
                 for (int r = 0; r < NR; ++r) {
-                    float v = sv[r];
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                    const float v = warp_max_f32(sv[r]);
                     if (lane == 0) rmax[warp * NR + r] = v;
                 }
                 if (bar_red_or(kNbRed, kSoftThreads, !ok || *abort_flag != 0)) {
