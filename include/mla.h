@@ -212,9 +212,10 @@ mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int32_t* bloc
  * mla_decode_workspace_bytes -- device workspace mla_decode needs for these
  * sizes (num_splits as passed to mla_decode; 0 = automatic).  It holds the
  * attend phase's pieces (a slot of 128 rows x (512 fp32 + max, sum) per
- * sequence plus one per CTA pair of the group, for each group of 128 query
- * rows; with G groups a group gets at most max(1, 74 / G) pairs) and the
- * merged latent output in bf16 ([H, ~B*n_q, 512]).
+ * sequence plus one per work unit of the group, for each group of 128 query
+ * rows; with G groups a group gets at most max(1, 74 / G) CTA pairs, and with
+ * n_q * H <= 32 the one group gets up to 148 one-SM units) and the merged
+ * latent output in bf16 ([H, ~B*n_q, 512]).
  */
 size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
 
@@ -248,7 +249,8 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
  * max_blocks * 128 sets MLA_DEVERR_ROW_RANGE; neither is processed and their
  * rows get out = 0 and lse = -inf.  A table entry outside [0, cap_blocks) sets
  * MLA_DEVERR_ROW_RANGE (that sequence's rows are then unspecified).
- * The call launches the attend kernel, then the merge and up-projection
+ * The call launches the attend kernel (CTA pairs; for n_q * H <= 32 a kernel
+ * that does a whole block on one SM), then the merge and up-projection
  * kernels (mla_decode_finish), each with programmatic stream serialization:
  * a kernel's set-up may overlap the end of the previous kernel on `stream`,
  * and it waits for that kernel to complete before reading any input.
