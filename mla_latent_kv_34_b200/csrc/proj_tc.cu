@@ -253,9 +253,9 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
     const int r = tid / kSplit, k = tid % kSplit;
-    grid_dependency_wait();  // the pieces come from the attend kernel
-    grid_dependents_launch();
-    // tiles of all sequences (the attend kernel's range split depends on the total) and before b
+    // tiles of all sequences (the attend kernel's range split depends on the total) and before b.  The
+    // lengths are an input of the decode call, the same for both phases, so they are read before the wait
+    // for the attend kernel's pieces and this part overlaps its tail.
     int s_all = 0, s_pre = 0;
     for (int i = tid; i < B; i += kMergeThreads) {
         const int n = valid_seq_tiles(kv_len[i], n_q, max_blocks);
@@ -279,6 +279,8 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
         ts += red[1][w];
     }
     const int ntb = valid_seq_tiles(kv_len[b], n_q, max_blocks);
+    grid_dependency_wait();  // the pieces come from the attend kernel
+    grid_dependents_launch();
     const int R = n_q * H;
     const int rr = g * 128 + r;
     const bool row_ok = rr < R;  // (no early exit: the shuffles below need every lane)
