@@ -10,10 +10,11 @@
 // rebuild the keys and values, so it does less arithmetic only once a key is shared by more than
 // ~171 queries: causal chunks of more than ~340 tokens.
 //
-// Kernel 1 (decompress): one CTA per (head, 128-token cache block).  The block's eight latent
-// chunks (already in the swizzled K-major operand layout in HBM) are the A operand; W^UK_h and
-// W^UV_h chunks, stacked as one N = 256 B operand, stream through a four-stage ring.  D[token,
-// 0..255] = [k^C | v^C] lands in TMEM; each thread writes its token's two 256-byte rows.
+// Kernel 1 (decompress): persistent, one CTA per SM taking (head, 128-token cache block) units.  A
+// block's eight latent chunks (already in the swizzled K-major operand layout in HBM) are the A
+// operand; W^UK_h and W^UV_h chunks, stacked as one N = 256 B operand, stream through a four-stage
+// ring that runs on across units.  D[token, 0..255] = [k^C | v^C] lands in one of two TMEM
+// accumulators; each thread writes its token's two 256-byte rows while the next unit's MMAs run.
 //
 // Kernel 2 (attend): one CTA per (head, 128-query tile).  Q [128 x 192] sits in shared memory;
 // key tiles (k^C by TMA from the workspace, k^R straight from the cache block's RoPE chunk, v^C by
@@ -66,7 +67,12 @@ constexpr int kDStageBytes = 3 * kChunk;  // cache chunk (A) + W^UK_h chunk + W^
 constexpr int kDStages = 4;
 constexpr int kDOffBar = kDStages * kDStageBytes;
 constexpr int kDSmemBytes = kDOffBar + 256;
+constexpr int kDMaxCtas = 148;  // one persistent CTA per SM
 
+// Persistent: CTA i takes the (head, block) units i, i + gridDim.x, ... (unit u = head u / nblk, block
+// u % nblk, so consecutive units share a head's weights).  The ring of stages runs on across units, and
+// the two 256-column TMEM accumulators alternate, so one unit's epilogue overlaps the next unit's loads
+// and MMAs.
 __global__ void __launch_bounds__(kThreads, 1) decompress_kernel(
     const __grid_constant__ CUtensorMap uk_map, const __grid_constant__ CUtensorMap uv_map,
     const uint8_t* __restrict__ cache, int64_t cap_blocks, const int32_t* __restrict__ blocks, int L, int H,
@@ -76,11 +82,15 @@ __global__ void __launch_bounds__(kThreads, 1) decompress_kernel(
     const uint32_t sbase = smem_u32(smem);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDOffBar);
     uint64_t* empty = full + kDStages;
-    uint64_t* done = empty + kDStages;
+    uint64_t* acc_full = empty + kDStages;   // [2] the MMAs of a unit are done
+    uint64_t* acc_empty = acc_full + 2;      // [2] the epilogue has read a unit's accumulator
+    uint64_t* fin = acc_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kDOffBar + 128);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kDOffBar + 136);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x, blk = blockIdx.y;
+    const int nblk = (L + kBlockTokens - 1) / kBlockTokens;
+    const int units = H * nblk;
+    volatile int never = 0;
     if ((sbase & 1023u) != 0) {
         if (tid == 0) report(dev_status, MLA_DEVERR_TIMEOUT);
         return;
@@ -90,11 +100,15 @@ __global__ void __launch_bounds__(kThreads, 1) decompress_kernel(
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 128);
+        }
+        mbar_init(fin, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) tmem_alloc(tmem_slot, 256);
+    if (warp == 0) tmem_alloc(tmem_slot, 512);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -104,76 +118,105 @@ __global__ void __launch_bounds__(kThreads, 1) decompress_kernel(
     if (warp == 4 && lane == 0) {
         prefetch_tmap(&uk_map);
         prefetch_tmap(&uv_map);
-        const uint8_t* src = tile_block(cache, blocks, cap_blocks, blk, dev_status);
-        const uint64_t keep = l2_policy_evict_last();  // every head's CTA reads this block
-        for (int c = 0; c < KC; ++c) {
-            const int s = c % kDStages, n = c / kDStages;
-            if (n > 0 && !mbar_wait(&empty[s], (n - 1) & 1, abort_flag, kLimitNs)) {
-                *abort_flag = 1;
-                report(dev_status, MLA_DEVERR_TIMEOUT);
-                break;
+        const uint64_t keep = l2_policy_evict_last();  // every head's unit reads this block
+        uint32_t nc = 0;                                 // stages filled
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+            const int h = u / nblk, blk = u % nblk;
+            const uint8_t* src = tile_block(cache, blocks, cap_blocks, blk, dev_status);
+            for (int c = 0; c < KC; ++c, ++nc) {
+                const uint32_t s = nc % kDStages, n = nc / kDStages;
+                if (n > 0 && !mbar_wait(&empty[s], (n - 1) & 1u, abort_flag, kLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t st = sbase + s * kDStageBytes;
+                mbar_arrive_expect_tx(&full[s], kDStageBytes);
+                bulk_load_hint(st, src + c * kBlockChunk, kChunk, &full[s], keep);
+                tma_load_2d(st + kChunk, &uk_map, c * 64, h * 128, &full[s]);
+                tma_load_2d(st + 2 * kChunk, &uv_map, c * 64, h * 128, &full[s]);
             }
-            const uint32_t st = sbase + s * kDStageBytes;
-            mbar_arrive_expect_tx(&full[s], kDStageBytes);
-            bulk_load_hint(st, src + c * kBlockChunk, kChunk, &full[s], keep);
-            tma_load_2d(st + kChunk, &uk_map, c * 64, h * 128, &full[s]);
-            tma_load_2d(st + 2 * kChunk, &uv_map, c * 64, h * 128, &full[s]);
         }
+        if (!ok) {
+            *abort_flag = 1;
+            report(dev_status, MLA_DEVERR_TIMEOUT);
+        }
+        // let every issued copy land before the CTA can exit
+        for (uint32_t i = (nc > kDStages ? nc - kDStages : 0); i < nc; ++i)
+            mbar_wait(&full[i % kDStages], (i / kDStages) & 1u, &never, kLimitNs);
     } else if (warp == 5 && lane == 0) {
         // D[token, 0..127] = k^C, D[token, 128..255] = v^C: A = latent chunk (M = 128 tokens),
-        // B = [W^UK_h ; W^UV_h] rows (N = 256), both K-major
+        // B = [W^UK_h ; W^UV_h] rows (N = 256), both K-major; accumulator ab = unit count & 1
         constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, false);
-        for (int c = 0; c < KC; ++c) {
-            const int s = c % kDStages, n = c / kDStages;
-            if (!mbar_wait(&full[s], n & 1, abort_flag, kLimitNs)) {
-                *abort_flag = 1;
-                report(dev_status, MLA_DEVERR_TIMEOUT);
+        uint32_t nc = 0, i = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++i) {
+            const uint32_t ab = i & 1u;
+            ok = mbar_wait(&acc_empty[ab], ((i >> 1) & 1u) ^ 1u, abort_flag, kLimitNs);
+            tc_fence_after();
+            for (int c = 0; ok && c < KC; ++c, ++nc) {
+                const uint32_t s = nc % kDStages, n = nc / kDStages;
+                ok = mbar_wait(&full[s], n & 1u, abort_flag, kLimitNs);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t st = sbase + s * kDStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tmem + 256 * ab, sdesc_sw128(st + kk * 32, 16, 1024),
+                           sdesc_sw128(st + kChunk + kk * 32, 16, 1024), idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(smem_u32(&empty[s]));
+            }
+            if (ok) mma_commit(smem_u32(&acc_full[ab]));
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            report(dev_status, MLA_DEVERR_TIMEOUT);
+        }
+        mma_commit(smem_u32(fin));  // TMEM is freed only once every MMA issued above is done
+    } else if (warp < 4) {
+        uint32_t i = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
+            const int h = u / nblk, blk = u % nblk;
+            const uint32_t ab = i & 1u;
+            const bool ok = mbar_wait(&acc_full[ab], (i >> 1) & 1u, abort_flag, kLimitNs);
+            __syncwarp();
+            tc_fence_after();
+            if (!__all_sync(0xffffffffu, ok) || *abort_flag) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    report(dev_status, MLA_DEVERR_TIMEOUT);
+                }
                 break;
             }
-            tc_fence_after();
-            const uint32_t st = sbase + s * kDStageBytes;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tmem, sdesc_sw128(st + kk * 32, 16, 1024), sdesc_sw128(st + kChunk + kk * 32, 16, 1024), idesc,
-                       (c > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(smem_u32(&empty[s]));
-        }
-        mma_commit(smem_u32(done));
-    } else if (warp < 4) {
-        const bool ok = mbar_wait(done, 0, abort_flag, kLimitNs);
-        __syncwarp();
-        tc_fence_after();
-        if (__all_sync(0xffffffffu, ok) && !*abort_flag) {
             const int t = blk * kBlockTokens + 32 * warp + lane;  // token of this TMEM lane
             const bool valid = t < L;
             for (int half = 0; half < 2; ++half) {
                 uint16_t* dst = (half == 0 ? k_out : v_out) + (static_cast<int64_t>(t) * H + h) * kDh;
                 for (int j0 = 0; j0 < kDh; j0 += 32) {
                     uint32_t v[32];
-                    tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 128 * half + j0, v);
+                    tmem_ld32(tmem + 256 * ab + (static_cast<uint32_t>(32 * warp) << 16) + 128 * half + j0, v);
                     tmem_wait_ld();
                     if (valid) {
                         uint4* d4 = reinterpret_cast<uint4*>(dst + j0);
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            d4[u] = make_uint4(pack_bf16x2(f32_of(v[8 * u]), f32_of(v[8 * u + 1])),
-                                               pack_bf16x2(f32_of(v[8 * u + 2]), f32_of(v[8 * u + 3])),
-                                               pack_bf16x2(f32_of(v[8 * u + 4]), f32_of(v[8 * u + 5])),
-                                               pack_bf16x2(f32_of(v[8 * u + 6]), f32_of(v[8 * u + 7])));
+                        for (int q = 0; q < 4; ++q)
+                            d4[q] = make_uint4(pack_bf16x2(f32_of(v[8 * q]), f32_of(v[8 * q + 1])),
+                                               pack_bf16x2(f32_of(v[8 * q + 2]), f32_of(v[8 * q + 3])),
+                                               pack_bf16x2(f32_of(v[8 * q + 4]), f32_of(v[8 * q + 5])),
+                                               pack_bf16x2(f32_of(v[8 * q + 6]), f32_of(v[8 * q + 7])));
                     }
                 }
             }
-        } else if (lane == 0) {
-            report(dev_status, MLA_DEVERR_TIMEOUT);
+            tc_fence_before();
+            mbar_arrive(&acc_empty[ab]);
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
-        volatile int never = 0;
-        mbar_wait(done, 0, &never, kLimitNs);
+        mbar_wait(fin, 0, &never, kLimitNs);
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -508,8 +551,9 @@ cudaError_t launch_prefill_naive(const uint16_t* q_nope, const uint16_t* q_rope,
     e = cudaFuncSetAttribute(pf::attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kASmemBytes);
     if (e != cudaSuccess) return e;
     const int nblk = (L + kBlockTokens - 1) / kBlockTokens;
-    pf::decompress_kernel<<<dim3(H, nblk), pf::kThreads, pf::kDSmemBytes, stream>>>(uk, uv, cache, cap_blocks, blocks,
-                                                                                  L, H, k_rows, v_rows, dev_status);
+    const int units = H * nblk;
+    pf::decompress_kernel<<<units < pf::kDMaxCtas ? units : pf::kDMaxCtas, pf::kThreads, pf::kDSmemBytes, stream>>>(
+        uk, uv, cache, cap_blocks, blocks, L, H, k_rows, v_rows, dev_status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     pf::attend_kernel<<<dim3(H, (n + 127) / 128), pf::kThreads, pf::kASmemBytes, stream>>>(
