@@ -105,3 +105,21 @@ def test_both_oracle_arms_sample_the_same_way():
     c = bench.step_counts(cfg, L)
     assert np.isclose(r["full_step_s"], 4.0 / 4000 * c["sum_L"] * cfg.H)
     assert np.isclose(r["value"], c["step_bytes"] / r["full_step_s"] / 1e12)
+
+
+def test_packed_upload_buffer_holds_every_input_at_aligned_offsets():
+    """The end-to-end leg uploads a step's inputs as one buffer: every tensor keeps its dtype, shape and
+    bytes, and starts on a 256-byte boundary (the library needs 16)."""
+    g = torch.Generator().manual_seed(3)
+    like = {"c_kv": torch.randn((5, 512), generator=g).bfloat16(), "pos": torch.arange(7, dtype=torch.int32),
+            "q_rope": torch.randn((3, 2, 64), generator=g).bfloat16(), "seq_idx": torch.zeros(1, dtype=torch.int32)}
+    buf, views = bench.packed(torch, like, "cpu", False)
+    base = buf.data_ptr()
+    for k, t in like.items():
+        v = views[k]
+        assert v.dtype == t.dtype and v.shape == t.shape
+        assert (v.data_ptr() - base) % 256 == 0
+        v.copy_(t)
+    for k, t in like.items():  # no view overlaps another
+        assert torch.equal(views[k], t)
+    assert buf.numel() == sum((t.numel() * t.element_size() + 255) // 256 * 256 for t in like.values())
