@@ -211,9 +211,9 @@ mla_status mla_append_cache(void* cache, int64_t cap_blocks, const int32_t* bloc
 /*
  * mla_decode_workspace_bytes -- device workspace mla_decode needs for these
  * sizes (num_splits as passed to mla_decode; 0 = automatic).  It holds the
- * attend phase's pieces (a slot of 128 rows x (512 fp32 + max, sum) per
- * sequence plus one per work unit of the group, for each group of 128 query
- * rows; with G groups a group gets at most max(1, 74 / G) CTA pairs, and with
+ * attend phase's pieces (a slot of 128 rows -- 32 when n_q * H <= 32 -- x
+ * (512 fp32 + max, sum) per sequence plus one per work unit of the group, for
+ * each group of 128 query rows; with G groups a group gets at most max(1, 74 / G) CTA pairs, and with
  * n_q * H <= 32 the one group gets up to 148 one-SM units) and the merged
  * latent output in bf16 ([H, ~B*n_q, 512]).
  */
@@ -295,7 +295,8 @@ mla_status mla_decode_finish(const int32_t* kv_len, int max_blocks, const void* 
  *   Arguments, layouts and results are those of mla_decode.
  *   Limit: shapes with mla_decode_workspace_bytes(B, n_q, H, num_splits) >
  *   MLA_DECODE_STATIC_SCRATCH_BYTES return MLA_ERR_WORKSPACE and launch
- *   nothing (for example B <= 32 at H = 128, n_q = 1).
+ *   nothing (for example B <= 32 at H = 128, n_q = 1; with n_q * H <= 32 the
+ *   slots are a quarter the size, so B = 64 fits at H = 16, n_q = 2).
  *   Set-up: the first call on a device looks the buffer up (and may load the
  *   library's device code there); make it before any stream capture.  The
  *   address found is kept for the life of the process: after a reset of the

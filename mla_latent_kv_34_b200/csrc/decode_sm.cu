@@ -83,12 +83,12 @@ struct Params {
     const uint8_t* cache;
     const int32_t* block_table;
     const int32_t* kv_len;
-    float* o_part;    // [slots][128 column groups of 4][128 rows] x float4
-    float2* ml_part;  // [slots][128]
+    float* o_part;    // [slots][128 column groups of 4][rs rows] x float4
+    float2* ml_part;  // [slots][rs]
     int32_t* dev_status;
     int64_t cap_blocks;
     int max_blocks;
-    int B, n_q, H, R, P_g, slots;
+    int B, n_q, H, R, P_g, slots, rs;
     float scale_log2;
 };
 
@@ -521,11 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm_kernel(const Params p) 
                 for (int r = 0; r < NR; ++r)
                     if (r == tk) mm = m[r];
                 const float l = rsum[tk] + rsum[NR + tk] + rsum[2 * NR + tk] + rsum[3 * NR + tk];
-                p.ml_part[static_cast<int64_t>(s.slot) * 128 + tk] = make_float2(mm, l);
+                p.ml_part[static_cast<int64_t>(s.slot) * p.rs + tk] = make_float2(mm, l);
             }
             // O^T: lane = latent column c = 128 mb + 32 warp + lane, column r = row; the workspace holds
-            // [column group c / 4][row] x float4
-            float* oseg = p.o_part + static_cast<int64_t>(s.slot) * 128 * kDc;
+            // [column group c / 4][row] x float4, rs rows per slot
+            float* oseg = p.o_part + static_cast<int64_t>(s.slot) * p.rs * kDc;
 #pragma unroll 1
             for (int mb = 0; mb < 4; ++mb) {
                 float v[NR];
@@ -533,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm_kernel(const Params p) 
                 const int c = 128 * mb + 32 * warp + lane;
 #pragma unroll
                 for (int r = 0; r < NR; ++r)
-                    if (r < p.R) oseg[((c >> 2) * 128 + r) * 4 + (c & 3)] = v[r];
+                    if (r < p.R) oseg[((c >> 2) * p.rs + r) * 4 + (c & 3)] = v[r];
             }
             tc_fence_before();
             mbar_arrive(&bars[kBOFree]);
@@ -601,9 +601,11 @@ int decode_sm_ctas() {
 
 cudaError_t launch_decode_sm(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
                              int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale, int ctas,
-                             float* o_part, float2* ml_part, int slots, int32_t* dev_status, cudaStream_t stream) {
+                             float* o_part, float2* ml_part, int slots, int rs, int32_t* dev_status,
+                             cudaStream_t stream) {
     const int R = n_q * H;
-    if (R < 1 || R > kMaxSmRows || ctas < 1 || ctas > kMaxSmCtas || B + ctas > slots) return cudaErrorInvalidValue;
+    if (R < 1 || R > kMaxSmRows || R > rs || ctas < 1 || ctas > kMaxSmCtas || B + ctas > slots)
+        return cudaErrorInvalidValue;
     sm1::Params prm;
     prm.q = q;
     prm.cache = cache;
@@ -620,6 +622,7 @@ cudaError_t launch_decode_sm(const uint16_t* q, const uint8_t* cache, int64_t ca
     prm.R = R;
     prm.P_g = ctas;
     prm.slots = slots;
+    prm.rs = rs;
     prm.scale_log2 = scale * 1.44269504088896340736f;
     return R <= 16 ? sm1::launch<16>(prm, stream) : sm1::launch<32>(prm, stream);
 }

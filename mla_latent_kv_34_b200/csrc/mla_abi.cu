@@ -39,12 +39,12 @@ int max_pairs_per_group(int G) { return kMaxPairs / G > 1 ? kMaxPairs / G : 1; }
 // Few query rows (n_q * H <= 32): the one-SM kernel (one row group, up to kMaxSmCtas CTAs) instead of CTA pairs.
 bool one_sm_path(int n_q, int H) { return static_cast<int64_t>(n_q) * H <= kMaxSmRows; }
 
-// ---- tensor-core path: segment partials [G][slots][128 rows] float2 (m, l), then (1024-aligned)
-//      [G][slots] blocks of 128 rows x 512 fp32 O, each stored as [128 column groups of 4][128 rows] x float4,
+// ---- tensor-core path: segment partials [G][slots][rs rows] float2 (m, l), then (1024-aligned)
+//      [G][slots] blocks of rs rows x 512 fp32 O, each stored as [128 column groups of 4][rs rows] x float4,
 //      then (1024-aligned) the merged latent output o_lat as bf16 operand tiles, [H][olat_rows(T)] x 1 KB.
 //      A slot per (sequence + CTA pair of the group): a pair's range starts at most one piece into a sequence.
 struct TcWs {
-    int G, slots;
+    int G, slots, rs;  // rs: rows per slot (128; kMaxSmRows on the one-SM path)
     size_t ml_part, o_part, olat, total;
 };
 
@@ -56,7 +56,8 @@ TcWs tc_ws_layout(int B, int n_q, int H) {
     // a group gets at most max(1, kMaxPairs / G) CTA pairs (long query chunks: many groups, few pairs each);
     // with few query rows the one-SM kernel's up to kMaxSmCtas CTAs share the single group
     w.slots = B + (one_sm_path(n_q, H) ? kMaxSmCtas : max_pairs_per_group(w.G));
-    const size_t rows = static_cast<size_t>(w.G) * w.slots * 128;
+    w.rs = one_sm_path(n_q, H) ? kMaxSmRows : 128;
+    const size_t rows = static_cast<size_t>(w.G) * w.slots * w.rs;
     w.ml_part = 0;
     w.o_part = align1k(rows * sizeof(float2));
     w.olat = align1k(w.o_part + rows * kDc * sizeof(float));
@@ -220,8 +221,8 @@ mla_status mla_decode_attend(const void* q, const void* cache, int64_t cap_block
         return cuda_status(launch_decode_sm(static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(cache),
                                             cap_blocks, block_table, max_blocks, kv_len, B, n_q, H, scale, pg,
                                             reinterpret_cast<float*>(ws + lay.o_part),
-                                            reinterpret_cast<float2*>(ws + lay.ml_part), lay.slots, dev_status,
-                                            static_cast<cudaStream_t>(stream)));
+                                            reinterpret_cast<float2*>(ws + lay.ml_part), lay.slots, lay.rs,
+                                            dev_status, static_cast<cudaStream_t>(stream)));
     return cuda_status(launch_decode_tc(static_cast<const uint16_t*>(q), static_cast<const uint8_t*>(cache),
                                         cap_blocks, block_table, max_blocks, kv_len, B, n_q, H, scale, pg,
                                         reinterpret_cast<float*>(ws + lay.o_part),
@@ -245,7 +246,8 @@ mla_status mla_decode_finish(const int32_t* kv_len, int max_blocks, const void* 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_merge(reinterpret_cast<const float*>(ws + lay.o_part),
                                  reinterpret_cast<const float2*>(ws + lay.ml_part), kv_len, max_blocks, B, n_q, H, pg,
-                                 lay.slots, reinterpret_cast<uint8_t*>(ws + lay.olat), lse_out, dev_status, cs);
+                                 lay.slots, lay.rs, reinterpret_cast<uint8_t*>(ws + lay.olat), lse_out, dev_status,
+                                 cs);
     if (e != cudaSuccess) return MLA_ERR_CUDA;
     return cuda_status(launch_upproj(reinterpret_cast<const uint8_t*>(ws + lay.olat),
                                      static_cast<const uint16_t*>(W_UV), B * n_q, H, static_cast<uint16_t*>(out),

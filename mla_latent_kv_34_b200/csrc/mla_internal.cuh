@@ -97,7 +97,8 @@ int decode_tc_clusters();
 int decode_sm_ctas();
 cudaError_t launch_decode_sm(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
                              int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale, int ctas,
-                             float* o_part, float2* ml_part, int slots, int32_t* dev_status, cudaStream_t stream);
+                             float* o_part, float2* ml_part, int slots, int rs, int32_t* dev_status,
+                             cudaStream_t stream);
 cudaError_t launch_decode_tc(const uint16_t* q, const uint8_t* cache, int64_t cap_blocks, const int32_t* block_table,
                              int max_blocks, const int32_t* kv_len, int B, int n_q, int H, float scale,
                              int clusters_per_group, float* o_part, float2* ml_part, int slots, int32_t* dev_status,
@@ -109,8 +110,8 @@ __host__ __device__ __forceinline__ int olat_rows(int T) {
     return full + ((rest + 15) / 16) * 16;
 }
 cudaError_t launch_merge(const float* o_part, const float2* ml_part, const int32_t* kv_len, int max_blocks, int B,
-                         int n_q, int H, int P_g, int slots, uint8_t* olat, float* lse_out, int32_t* dev_status,
-                         cudaStream_t stream);
+                         int n_q, int H, int P_g, int slots, int rs, uint8_t* olat, float* lse_out,
+                         int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_upproj(const uint8_t* olat, const uint16_t* W_UV, int T, int H, uint16_t* out, int32_t* dev_status,
                           cudaStream_t stream);
 

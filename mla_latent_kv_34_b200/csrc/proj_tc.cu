@@ -247,7 +247,8 @@ __device__ __forceinline__ int64_t olat_offset(int T, int h, int t, int c, int u
 template <int kSplit>
 __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
     const float* __restrict__ o_part, const float2* __restrict__ ml_part, const int32_t* __restrict__ kv_len,
-    int max_blocks, int B, int n_q, int H, int P_g, int slots, uint8_t* __restrict__ olat, float* __restrict__ lse_out) {
+    int max_blocks, int B, int n_q, int H, int P_g, int slots, int rs, uint8_t* __restrict__ olat,
+    float* __restrict__ lse_out) {
     constexpr int kMergeThreads = 128 * kSplit;
     __shared__ int red[2][kMergeThreads / 32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -304,12 +305,12 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
     const int cg0 = 8 * slice;  // column groups 8 slice .. 8 slice + 7 = columns 32 slice .. + 31
     for (int p = p_first + k; p <= p_last; p += kSplit) {
         if (!live(p)) continue;
-        // segment partials: [column group of 4][128 rows] x float4; the loads go out before the (m, l) test
-        const float4* src = reinterpret_cast<const float4*>(o_part) + ((seg0 + p) * 128 + cg0) * 128 + r;
+        // segment partials: [column group of 4][rs rows] x float4; the loads go out before the (m, l) test
+        const float4* src = reinterpret_cast<const float4*>(o_part) + ((seg0 + p) * 128 + cg0) * rs + r;
         float4 v[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = src[i * 128];
-        const float2 ml = ml_part[(seg0 + p) * 128 + r];
+        for (int i = 0; i < 8; ++i) v[i] = src[i * rs];
+        const float2 ml = ml_part[(seg0 + p) * rs + r];
         if (ml.x == -CUDART_INF_F) continue;
         const float Mn = fmaxf(M, ml.x);
         const float sc = exp2f(M - Mn), w = exp2f(ml.x - Mn);
@@ -548,8 +549,8 @@ cudaError_t launch_absorb_tc(const uint16_t* q_nope, const uint16_t* q_rope, con
 }
 
 cudaError_t launch_merge(const float* o_part, const float2* ml_part, const int32_t* kv_len, int max_blocks, int B,
-                         int n_q, int H, int P_g, int slots, uint8_t* olat, float* lse_out, int32_t* dev_status,
-                         cudaStream_t stream) {
+                         int n_q, int H, int P_g, int slots, int rs, uint8_t* olat, float* lse_out,
+                         int32_t* dev_status, cudaStream_t stream) {
     (void)dev_status;
     const int G = (n_q * H + 127) / 128;
     const dim3 grid(proj::kMergeSlices, B, G);
@@ -557,12 +558,12 @@ cudaError_t launch_merge(const float* o_part, const float2* ml_part, const int32
     const int per = P_g / (B > 0 ? B : 1);
     if (per >= 4)
         return proj::launch_pdl(proj::merge_kernel<4>, grid, 512, 0, stream, o_part, ml_part, kv_len, max_blocks, B,
-                                n_q, H, P_g, slots, olat, lse_out);
+                                n_q, H, P_g, slots, rs, olat, lse_out);
     if (per >= 1)
         return proj::launch_pdl(proj::merge_kernel<2>, grid, 256, 0, stream, o_part, ml_part, kv_len, max_blocks, B,
-                                n_q, H, P_g, slots, olat, lse_out);
+                                n_q, H, P_g, slots, rs, olat, lse_out);
     return proj::launch_pdl(proj::merge_kernel<1>, grid, 128, 0, stream, o_part, ml_part, kv_len, max_blocks, B, n_q,
-                            H, P_g, slots, olat, lse_out);
+                            H, P_g, slots, rs, olat, lse_out);
 }
 
 cudaError_t launch_upproj(const uint8_t* olat, const uint16_t* W_UV, int T, int H, uint16_t* out, int32_t* dev_status,

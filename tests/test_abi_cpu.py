@@ -123,22 +123,23 @@ def test_host_validation_rejects_bad_arguments(mla):
 def test_workspace_sizes(mla):
     # tensor-core path: one slot per (sequence + work unit) and row group, any split count, plus the merged
     # latent output (bf16, rows rounded up to a multiple of 16).  Work units: CTA pairs (at most 74 / G per
-    # group), or with at most 32 query rows the one-SM kernel's CTAs (at most 148, one group)
+    # group; 128 rows per slot), or with at most 32 query rows the one-SM kernel's CTAs (at most 148, one
+    # group; 32 rows per slot)
     a = mla.decode_workspace_bytes(32, 1, 128, 1)
     assert a == mla.decode_workspace_bytes(32, 1, 128, 0) > 32 * 128 * 512 * 4
     assert mla.decode_workspace_bytes(32, 2, 128, 0) > a  # two row groups, 37 pairs each (exact sizes below)
-    slot = 128 * (8 + 512 * 4)
     for B, n_q, H in [(32, 1, 128), (128, 2, 128), (1, 1, 16), (70, 1, 3), (1, 256, 128), (3, 100, 16),
                       (64, 1, 16), (5, 2, 16), (5, 3, 11), (2, 1, 33)]:
         G = (n_q * H + 127) // 128
         units = 148 if n_q * H <= 32 else max(1, 74 // G)
-        rows = G * (B + units) * 128
+        rs = 32 if n_q * H <= 32 else 128  # rows per slot
+        rows = G * (B + units) * rs
         T = B * n_q
         olat_rows = (T + 15) // 16 * 16
         head = -(-rows * 8 // 1024) * 1024
         want = -(-(head + rows * 512 * 4) // 1024) * 1024 + H * olat_rows * 1024
         assert mla.decode_workspace_bytes(B, n_q, H, 0) == want, (B, n_q, H)
-        assert want >= rows * slot // 128
+        assert want >= rows * (8 + 512 * 4)
     # CUDA-core path: one fp32 partial per split
     c1 = mla.lib.mla_decode_cudacore_workspace_bytes(32, 1, 128, 1)
     c4 = mla.lib.mla_decode_cudacore_workspace_bytes(32, 1, 128, 4)

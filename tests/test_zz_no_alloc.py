@@ -33,6 +33,11 @@ def test_no_alloc_limit_matches_the_library():
     st = mla.lib.mla_decode_static(None, None, 0, None, 0, None, None, 32, 1, 128, ctypes.c_float(0.07), 0,
                                    None, None, None, None)
     assert st == 1, mla.lib.mla_status_string(st).decode()
+    # few heads (the one-SM path, 32 rows per slot): a V2-Lite-sized batch fits as well
+    assert mla.decode_workspace_bytes(64, 1, 16) <= lim
+    st = mla.lib.mla_decode_static(None, None, 0, None, 0, None, None, 64, 1, 16, ctypes.c_float(0.07), 0,
+                                   None, None, None, None)
+    assert st == 1, mla.lib.mla_status_string(st).decode()
 
 
 @pytest.mark.gpu
@@ -85,3 +90,30 @@ def test_no_alloc_decode_at_the_scratch_limit_matches_oracle(cuda_ok):
         got = got_all[b][None][:, heads]
         assert np.all(np.abs(got - ref) <= ATOL + RTOL * np.abs(ref)), f"seq {b}"
         assert np.abs(lse_all[b][heads] - ref_lse[0]).max() < 2e-2
+
+
+@pytest.mark.gpu
+def test_no_alloc_decode_few_heads_matches_oracle(cuda_ok):
+    """Few heads (n_q * H <= 32: the one-SM attend kernel, 32 rows per workspace slot) through the
+    library-owned scratch: the same result as mla_decode and the oracle on sampled sequences."""
+    import gpu_harness as H
+    import mla_latent_kv_34_b200 as mla
+    cfg = mi.MLAConfig("no-alloc-few", B=64, H=16, n_q=2, L=None, L_max=900, seed=93)
+    assert mla.decode_workspace_bytes(cfg.B, cfg.n_q, cfg.H) <= mla.DECODE_STATIC_SCRATCH_BYTES
+    prob = H.build_problem(cfg, shuffle_seed=4)
+    q = prob.absorb()
+    ref, ref_lse = prob.decode(q)
+    out = torch.empty_like(ref)
+    lse = torch.empty_like(ref_lse)
+    mla.decode_static(q, prob.cache, prob.block_table, prob.kv_len, prob.W_UV, cfg.n_q, cfg.scale,
+                      out=out, lse_out=lse, dev_status=prob.status)
+    torch.cuda.synchronize()
+    assert int(prob.status.item()) == 0
+    a, b = out.float().cpu().numpy(), ref.float().cpu().numpy()
+    assert np.all(np.abs(a - b) <= ATOL + RTOL * np.abs(b))
+    got_all = a.reshape(cfg.B, cfg.n_q, cfg.H, 128)
+    lse_all = lse.cpu().numpy().reshape(cfg.B, cfg.n_q, cfg.H)
+    for bb in (0, 31, 63):
+        ref_o, _, ref_l = prob.oracle(bb)
+        assert np.all(np.abs(got_all[bb] - ref_o) <= ATOL + RTOL * np.abs(ref_o)), f"seq {bb}"
+        assert np.abs(lse_all[bb] - ref_l).max() < 2e-2
