@@ -224,8 +224,6 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
 
 // ------------------------------------------------------------------ merge
 
-constexpr int kMergeSlices = 16;    // a CTA merges 32 of the 512 latent columns (8 column groups of 4)
-
 // Byte offset of row t of head h, latent unit (chunk c, unit u) in the o_lat tiles: per head, the rows
 // are cut into blocks of kOlatBlock (the last one olat_rows(T) - kOlatBlock * (blocks - 1) rows); a block
 // is eight [rows x 64] chunks, each 128-byte swizzled, so chunk c of a block is the K-major B operand of
@@ -238,27 +236,32 @@ __device__ __forceinline__ int64_t olat_offset(int T, int h, int t, int c, int u
     return (static_cast<int64_t>(h) * Tp + kOlatBlock * tb) * 1024 + c * rows * 128 + swz(i, u);
 }
 
-// One CTA per (32-column slice, sequence, row group).  Row r of the group is merged by kSplit threads
-// (neighbouring lanes), each over every kSplit-th piece of the sequence with its own running maximum; their
-// partial results are combined with warp shuffles.  kSplit follows the expected pieces per sequence (1 when
-// sequences outnumber the CTA pairs, up to 4 for a few long sequences cut into many pieces).  A thread's
-// loads of one piece are eight 16-byte column groups of its row (the attend kernel's [column group][row]
-// order).
-template <int kSplit>
-__global__ void __launch_bounds__(128 * kSplit) merge_kernel(
+// One CTA per (column slice, sequence, row group); blockDim = rows x kSplit with rows = min(128, rows per slot).
+// Row r of the group is merged by kSplit threads (neighbouring lanes), each over every kSplit-th piece of the
+// sequence with its own running maximum; their partial results are combined with warp shuffles.  A thread
+// covers kVec column groups of 4 (slice = 4 kVec columns, 128 / kVec slices per row) and issues the loads of
+// 8 / kVec pieces before it uses any, so that every thread has eight 16-byte loads in flight per round trip.
+// The launch picks kSplit from the expected pieces per sequence and kVec from the number of CTAs, so that a
+// few long sequences cut into many pieces still spread over the whole GPU.  A thread's loads of one piece
+// are kVec 16-byte column groups of its row (the attend kernel's [column group][row] order).
+template <int kSplit, int kVec>
+__global__ void __launch_bounds__(512) merge_kernel(
     const float* __restrict__ o_part, const float2* __restrict__ ml_part, const int32_t* __restrict__ kv_len,
     int max_blocks, int B, int n_q, int H, int P_g, int slots, int rs, uint8_t* __restrict__ olat,
     float* __restrict__ lse_out) {
-    constexpr int kMergeThreads = 128 * kSplit;
-    __shared__ int red[2][kMergeThreads / 32];
+    static_assert(kSplit >= 1 && kSplit <= 32 && (kSplit & (kSplit - 1)) == 0, "kSplit: power of two <= 32");
+    static_assert(kVec == 2 || kVec == 4 || kVec == 8, "kVec: 2, 4 or 8 column groups");
+    constexpr int kBatch = 8 / kVec;  // pieces whose loads are in flight together
+    __shared__ int red[2][16];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nthr = blockDim.x, nwarps = nthr >> 5;
     const int slice = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
     const int r = tid / kSplit, k = tid % kSplit;
     // tiles of all sequences (the attend kernel's range split depends on the total) and before b.  The
     // lengths are an input of the decode call, the same for both phases, so they are read before the wait
     // for the attend kernel's pieces and this part overlaps its tail.
     int s_all = 0, s_pre = 0;
-    for (int i = tid; i < B; i += kMergeThreads) {
+    for (int i = tid; i < B; i += nthr) {
         const int n = valid_seq_tiles(kv_len[i], n_q, max_blocks);
         s_all += n;
         if (i < b) s_pre += n;
@@ -274,8 +277,7 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
     }
     __syncthreads();
     int Nt = 0, ts = 0;
-#pragma unroll
-    for (int w = 0; w < kMergeThreads / 32; ++w) {
+    for (int w = 0; w < nwarps; ++w) {
         Nt += red[0][w];
         ts += red[1][w];
     }
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
     grid_dependents_launch();
     const int R = n_q * H;
     const int rr = g * 128 + r;
-    const bool row_ok = rr < R;  // (no early exit: the shuffles below need every lane)
+    const bool row_ok = r < rs && rr < R;  // (no early exit: the shuffles below need every lane)
     // pieces of sequence b: the attend kernel's pairs whose tile range [lo, hi) meets [ts, ts + ntb)
     int p_first = 0, p_last = -1;
     if (ntb > 0 && Nt > 0 && row_ok) {
@@ -299,29 +301,40 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
         return max(lo, ts) < min(hi, ts + ntb);
     };
     float M = -CUDART_INF_F, z = 0.f;
-    float acc[32];
+    float acc[4 * kVec];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-    const int cg0 = 8 * slice;  // column groups 8 slice .. 8 slice + 7 = columns 32 slice .. + 31
-    for (int p = p_first + k; p <= p_last; p += kSplit) {
-        if (!live(p)) continue;
-        // segment partials: [column group of 4][rs rows] x float4; the loads go out before the (m, l) test
-        const float4* src = reinterpret_cast<const float4*>(o_part) + ((seg0 + p) * 128 + cg0) * rs + r;
-        float4 v[8];
+    for (int i = 0; i < 4 * kVec; ++i) acc[i] = 0.f;
+    const int cg0 = kVec * slice;  // column groups cg0 .. cg0 + kVec - 1 = columns 4 cg0 .. 4 cg0 + 4 kVec - 1
+    for (int p0 = p_first + k; p0 <= p_last; p0 += kSplit * kBatch) {
+        // segment partials: [column group of 4][rs rows] x float4; every load of the batch goes out before
+        // the (m, l) tests
+        float4 v[kBatch][kVec];
+        float2 ml[kBatch];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = src[i * rs];
-        const float2 ml = ml_part[(seg0 + p) * rs + r];
-        if (ml.x == -CUDART_INF_F) continue;
-        const float Mn = fmaxf(M, ml.x);
-        const float sc = exp2f(M - Mn), w = exp2f(ml.x - Mn);
-        z = z * sc + ml.y * w;
-        M = Mn;
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * kSplit;
+            ml[u] = make_float2(-CUDART_INF_F, 0.f);
+            if (p <= p_last && live(p)) {
+                const float4* src = reinterpret_cast<const float4*>(o_part) + ((seg0 + p) * 128 + cg0) * rs + r;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            acc[4 * i] = fmaf(w, v[i].x, acc[4 * i] * sc);
-            acc[4 * i + 1] = fmaf(w, v[i].y, acc[4 * i + 1] * sc);
-            acc[4 * i + 2] = fmaf(w, v[i].z, acc[4 * i + 2] * sc);
-            acc[4 * i + 3] = fmaf(w, v[i].w, acc[4 * i + 3] * sc);
+                for (int i = 0; i < kVec; ++i) v[u][i] = src[i * rs];
+                ml[u] = ml_part[(seg0 + p) * rs + r];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            if (ml[u].x == -CUDART_INF_F) continue;
+            const float Mn = fmaxf(M, ml[u].x);
+            const float sc = exp2f(M - Mn), w = exp2f(ml[u].x - Mn);
+            z = z * sc + ml[u].y * w;
+            M = Mn;
+#pragma unroll
+            for (int i = 0; i < kVec; ++i) {
+                acc[4 * i] = fmaf(w, v[u][i].x, acc[4 * i] * sc);
+                acc[4 * i + 1] = fmaf(w, v[u][i].y, acc[4 * i + 1] * sc);
+                acc[4 * i + 2] = fmaf(w, v[u][i].z, acc[4 * i + 2] * sc);
+                acc[4 * i + 3] = fmaf(w, v[u][i].w, acc[4 * i + 3] * sc);
+            }
         }
     }
     // combine the row's kSplit partial merges (neighbouring lanes)
@@ -333,7 +346,7 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
 #pragma unroll
     for (int o = 1; o < kSplit; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < 4 * kVec; ++i) {
         float a = acc[i] * sc;
 #pragma unroll
         for (int o = 1; o < kSplit; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
@@ -344,18 +357,18 @@ __global__ void __launch_bounds__(128 * kSplit) merge_kernel(
     const int t = b * n_q + j;
     const int T = B * n_q;
     const float inv = (z > 0.f) ? 1.f / z : 0.f;
-    // columns 32 slice .. + 31 = chunk slice / 2, units 4 (slice & 1) .. + 3; thread k writes the units
-    // q with q % kSplit == k (16 bytes = columns 8 q .. 8 q + 7 of the slice)
-    const int c = slice >> 1;
+    // the slice's kVec / 2 units of 8 columns (16 bytes of bf16); thread k writes the units q with
+    // q % kSplit == k.  Column 4 cg0 + 8 q is in chunk (4 cg0 + 8 q) / 64, unit ((4 cg0 + 8 q) % 64) / 8.
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kVec / 2; ++q) {
         if (q % kSplit != k) continue;
+        const int col = 4 * cg0 + 8 * q;
         uint4 y;
         y.x = pack_bf16x2(acc[8 * q] * inv, acc[8 * q + 1] * inv);
         y.y = pack_bf16x2(acc[8 * q + 2] * inv, acc[8 * q + 3] * inv);
         y.z = pack_bf16x2(acc[8 * q + 4] * inv, acc[8 * q + 5] * inv);
         y.w = pack_bf16x2(acc[8 * q + 6] * inv, acc[8 * q + 7] * inv);
-        *reinterpret_cast<uint4*>(olat + olat_offset(T, h, t, c, 4 * (slice & 1) + q)) = y;
+        *reinterpret_cast<uint4*>(olat + olat_offset(T, h, t, col >> 6, (col & 63) >> 3)) = y;
     }
     if (slice == 0 && k == 0 && lse_out)
         lse_out[static_cast<int64_t>(t) * H + h] = (z > 0.f) ? (Mr + log2f(z)) * 0.69314718055994530942f : -CUDART_INF_F;
@@ -548,22 +561,61 @@ cudaError_t launch_absorb_tc(const uint16_t* q_nope, const uint16_t* q_rope, con
                             q_rope, pos, rope_table, rope_len, T, H, q_out, dev_status);
 }
 
+namespace proj {
+
+template <int kSplit, int kVec>
+cudaError_t launch_merge_t(int rows, dim3 grid, cudaStream_t stream, const float* o_part, const float2* ml_part,
+                           const int32_t* kv_len, int max_blocks, int B, int n_q, int H, int P_g, int slots, int rs,
+                           uint8_t* olat, float* lse_out) {
+    grid.x = 128 / kVec;
+    return launch_pdl(merge_kernel<kSplit, kVec>, grid, rows * kSplit, 0, stream, o_part, ml_part, kv_len,
+                      max_blocks, B, n_q, H, P_g, slots, rs, olat, lse_out);
+}
+
+template <int kSplit>
+cudaError_t launch_merge_s(int vec, int rows, dim3 grid, cudaStream_t stream, const float* o_part,
+                           const float2* ml_part, const int32_t* kv_len, int max_blocks, int B, int n_q, int H,
+                           int P_g, int slots, int rs, uint8_t* olat, float* lse_out) {
+    if (vec == 8)
+        return launch_merge_t<kSplit, 8>(rows, grid, stream, o_part, ml_part, kv_len, max_blocks, B, n_q, H, P_g,
+                                         slots, rs, olat, lse_out);
+    if (vec == 4)
+        return launch_merge_t<kSplit, 4>(rows, grid, stream, o_part, ml_part, kv_len, max_blocks, B, n_q, H, P_g,
+                                         slots, rs, olat, lse_out);
+    return launch_merge_t<kSplit, 2>(rows, grid, stream, o_part, ml_part, kv_len, max_blocks, B, n_q, H, P_g, slots,
+                                     rs, olat, lse_out);
+}
+
+}  // namespace proj
+
 cudaError_t launch_merge(const float* o_part, const float2* ml_part, const int32_t* kv_len, int max_blocks, int B,
                          int n_q, int H, int P_g, int slots, int rs, uint8_t* olat, float* lse_out,
                          int32_t* dev_status, cudaStream_t stream) {
     (void)dev_status;
+    if (B < 1 || rs < 1 || rs > 128 || (rs & 31) != 0) return cudaErrorInvalidValue;
     const int G = (n_q * H + 127) / 128;
-    const dim3 grid(proj::kMergeSlices, B, G);
-    // pieces per sequence ~ 1 + P_g / B: one thread per row when sequences outnumber the pairs
-    const int per = P_g / (B > 0 ? B : 1);
-    if (per >= 4)
-        return proj::launch_pdl(proj::merge_kernel<4>, grid, 512, 0, stream, o_part, ml_part, kv_len, max_blocks, B,
-                                n_q, H, P_g, slots, rs, olat, lse_out);
-    if (per >= 1)
-        return proj::launch_pdl(proj::merge_kernel<2>, grid, 256, 0, stream, o_part, ml_part, kv_len, max_blocks, B,
-                                n_q, H, P_g, slots, rs, olat, lse_out);
-    return proj::launch_pdl(proj::merge_kernel<1>, grid, 128, 0, stream, o_part, ml_part, kv_len, max_blocks, B, n_q,
-                            H, P_g, slots, rs, olat, lse_out);
+    const int rows = rs;  // rows per slot: 128, or 32 for the one-SM kernel's pieces
+    // Threads per row: enough that none merges more than about five pieces (a sequence has about 1 + P_g / B
+    // of them); then slices as wide as possible while the grid still has 64 K threads.  Measured at V2, 128K
+    // and V2-Lite shapes (in a step, after the attend kernel), wider or narrower choices were slower: more
+    // threads per row mostly add CTAs that wait, and narrow slices multiply the sequence-length prologue.
+    int split = 1;
+    while (split < 16 && rows * split * 2 <= 512 && static_cast<int64_t>(B) + P_g > int64_t(5) * split * B) split *= 2;
+    int vec = 8;
+    while (vec > 2 && int64_t(128 / vec) * B * G * rows * split < 65536) vec /= 2;
+    const dim3 grid(1, B, G);
+    switch (split) {
+        case 1: return proj::launch_merge_s<1>(vec, rows, grid, stream, o_part, ml_part, kv_len, max_blocks, B, n_q,
+                                               H, P_g, slots, rs, olat, lse_out);
+        case 2: return proj::launch_merge_s<2>(vec, rows, grid, stream, o_part, ml_part, kv_len, max_blocks, B, n_q,
+                                               H, P_g, slots, rs, olat, lse_out);
+        case 4: return proj::launch_merge_s<4>(vec, rows, grid, stream, o_part, ml_part, kv_len, max_blocks, B, n_q,
+                                               H, P_g, slots, rs, olat, lse_out);
+        case 8: return proj::launch_merge_s<8>(vec, rows, grid, stream, o_part, ml_part, kv_len, max_blocks, B, n_q,
+                                               H, P_g, slots, rs, olat, lse_out);
+        default: return proj::launch_merge_s<16>(vec, rows, grid, stream, o_part, ml_part, kv_len, max_blocks, B,
+                                                 n_q, H, P_g, slots, rs, olat, lse_out);
+    }
 }
 
 cudaError_t launch_upproj(const uint8_t* olat, const uint16_t* W_UV, int T, int H, uint16_t* out, int32_t* dev_status,

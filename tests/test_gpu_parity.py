@@ -253,11 +253,13 @@ def test_decode_split_invariance(cuda_ok, H, splits):
 @pytest.mark.parametrize("B,Hh,n_q,L_max,splits,shuffle", [(7, 16, 2, 1500, 0, 3), (3, 4, 1, 700, 0, None),
                                                           (5, 11, 2, 2000, 3, 5), (1, 1, 1, 5, 0, None),
                                                           (40, 16, 1, 600, 1, 7), (6, 32, 1, 2600, 0, 9),
-                                                          (4, 16, 2, 300, 200, None)])
+                                                          (4, 16, 2, 300, 200, None), (20, 16, 1, 900, 0, 11),
+                                                          (100, 8, 2, 400, 0, 13)])
 def test_decode_few_rows_one_sm_kernel(cuda_ok, H, B, Hh, n_q, L_max, splits, shuffle):
     """At most 32 query rows (n_q * H): the one-SM kernel (tokens as the MMA's M side, both contractions on
     one SM), with shuffled block tables and NaN canaries in unowned blocks, against the CUDA-core path and
-    the oracle; one work unit per SM down to a single one, and more units than tiles."""
+    the oracle; one work unit per SM down to a single one, and more units than tiles.  The batch sizes
+    also take the merge through 1, 2, 8 and 16 threads per row."""
     cfg = mi.MLAConfig("one-sm", B=B, H=Hh, n_q=n_q, L=None, L_max=L_max, seed=700 + B + Hh + n_q)
     prob = H.build_problem(cfg, shuffle_seed=shuffle)
     q = prob.absorb()
