@@ -199,9 +199,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm_kernel(const Params p) 
     if (warp == kWarpProducer) tmem_alloc(tmem_slot, L::kTmemCols);
     // everything above touches only this CTA's own resources; inputs are read after this wait
     grid_dependency_wait();
-    // The merge kernel may be scheduled from here on: its CTAs take the SMs that this grid's CTAs leave,
-    // read the sequence lengths and then wait (in the hardware) for this whole grid to finish.
-    grid_dependents_launch();
     if (warp == 0) {
         // total tiles, then (by a warp scan) the sequence holding this CTA's first tile
         int s = 0;
@@ -547,6 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_sm_kernel(const Params p) 
     }
 
     // ------------------------------------------------------------------ teardown
+    grid_dependents_launch();  // the merge kernel may be scheduled; it waits for this grid to finish
     tc_fence_before();
     __syncthreads();
     if (warp == kWarpProducer) {

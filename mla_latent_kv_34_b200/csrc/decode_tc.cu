@@ -256,9 +256,6 @@ decode_tc_kernel(const Params p) {
     // Everything above touches only this CTA's own resources, so it overlaps the previous kernel's tail
     // under programmatic dependent launch; every read of the call's inputs comes after this wait.
     grid_dependency_wait();
-    // The merge kernel may be scheduled from here on: its CTAs take the SMs that this grid's CTAs leave,
-    // read the sequence lengths and then wait (in the hardware) for this whole grid to finish.
-    grid_dependents_launch();
     if (warp == 0) {
         // total tiles, then (by a warp scan) the sequence holding this cluster's first tile
         int s = 0;
@@ -812,6 +809,7 @@ decode_tc_kernel(const Params p) {
     }
 
     // ------------------------------------------------------------------ teardown
+    grid_dependents_launch();  // the merge kernel may be scheduled; it waits for this grid to finish
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // the peer no longer touches this CTA's shared memory

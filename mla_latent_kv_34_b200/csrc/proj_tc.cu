@@ -38,7 +38,6 @@ using namespace sm100;
 namespace proj {
 
 constexpr int kWChunkBytes = 128 * 64 * 2;   // [128 rows x 64 columns] bf16 = 16 KB
-constexpr int kWBytes = 8 * kWChunkBytes;    // one head's weight matrix, 128 KB
 constexpr int kTokBlock = 128;               // absorb: query rows per CTA (MMA N <= 128)
 constexpr uint64_t kLimitNs = 2000000000ull;
 
@@ -190,13 +189,18 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
         }
     }
     ok = __syncthreads_and(ok);
+    bool done = false;
     if (ok) {
-        // D: lane = latent column 128 mb + 32 warp + lane, column = row t
-        const bool done = mbar_wait(&bars[1], 0, &never, kLimitNs);
+        // D: lane = latent column 128 mb + 32 warp + lane, column = row t.  Once the MMAs are done the B
+        // operand's space is free: row j of the result goes there as 256 bytes of bf16, so that it leaves
+        // as 16-byte stores (a thread per column would store 2 bytes into each of 32 rows).
+        done = mbar_wait(&bars[1], 0, &never, kLimitNs);
         __syncwarp();
         tc_fence_after();
-        if (__all_sync(0xffffffffu, done)) {
-            const int c = 128 * mb + 32 * warp + lane;
+        done = __all_sync(0xffffffffu, done);
+        if (done) {
+            uint16_t* stage = reinterpret_cast<uint16_t*>(smem + kAbsOffB);
+            const int cl = 32 * warp + lane;
             for (int j0 = 0; j0 < NT; j0 += 32) {
                 uint32_t v[32];
                 const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + j0;
@@ -206,12 +210,18 @@ __global__ void __launch_bounds__(kAbsThreads) absorb_tc_kernel(
                 const int jn = min(32, nt - j0);
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    if (j < jn)
-                        q_out[(static_cast<int64_t>(t0 + j0 + j) * H + h) * kRow + c] =
-                            f32_to_bf16_rne(__uint_as_float(v[j]));
+                    if (j < jn) stage[(j0 + j) * 128 + cl] = f32_to_bf16_rne(__uint_as_float(v[j]));
             }
         } else if (lane == 0) {
             report(dev_status, MLA_DEVERR_TIMEOUT);
+        }
+    }
+    if (__syncthreads_and(done)) {
+        // rows t0 .. t0 + nt - 1, latent columns 128 mb .. 128 mb + 127: 16 units of 16 bytes per row
+        for (int idx = tid; idx < nt * 16; idx += kAbsThreads) {
+            const int j = idx >> 4, u = idx & 15;
+            const uint4 y = *reinterpret_cast<const uint4*>(smem + kAbsOffB + j * 256 + u * 16);
+            reinterpret_cast<uint4*>(q_out + (static_cast<int64_t>(t0 + j) * H + h) * kRow + 128 * mb)[u] = y;
         }
     }
     tc_fence_before();
@@ -377,33 +387,42 @@ __global__ void __launch_bounds__(512) merge_kernel(
 // ------------------------------------------------------------------ up-projection
 
 constexpr int kUpThreads = 128;
-constexpr int kUpRows = kOlatBlock;                        // o_lat rows per CTA = one o_lat block (MMA N <= 256)
-constexpr int kUpStages = 4;                               // ring of K chunks (8 per head)
-constexpr int kUpOffB = kWChunkBytes;                      // stage: W^UV chunk (16 KB) | o_lat chunk (<= 32 KB)
-constexpr int kUpStageBytes = kWChunkBytes + kUpRows * 128;
-constexpr int kUpOffBar = kUpStages * kUpStageBytes;
-constexpr int kUpSmemBytes = kUpOffBar + 128;
-static_assert(kUpStageBytes % 1024 == 0 && kUpRows * kDh * 2 <= kUpOffBar, "stages 1024-aligned; output staging fits");
 
-// One CTA per (head, block of up to 256 o_lat rows).  The contraction over the 512 latent columns streams
-// through a ring of four stages, one 64-column chunk per stage: W^UV_h's chunk as a [128 x 64] TMA box (the
+// Shared-memory plan of the up-projection: kStages stages of [W^UV chunk (16 KB) | o_lat chunk (kRows x 128 B)],
+// then the barriers (full[kStages], empty[kStages], done) and the TMEM address.
+template <int kRows, int kStages>
+struct UpPlan {
+    static constexpr int kOffB = kWChunkBytes;
+    static constexpr int kStageBytes = kWChunkBytes + kRows * 128;
+    static constexpr int kOffBar = kStages * kStageBytes;
+    static constexpr int kSmemBytes = kOffBar + 256;
+    static_assert(kStageBytes % 1024 == 0 && kRows * kDh * 2 <= kOffBar, "stages 1024-aligned; output staging fits");
+    static_assert(8 * (2 * kStages + 1) + 4 <= 256 && kSmemBytes <= 227 * 1024, "barriers and stages fit");
+};
+
+// One CTA per (head, block of up to kRows o_lat rows).  The contraction over the 512 latent columns streams
+// through a ring of kStages stages, one 64-column chunk per stage: W^UV_h's chunk as a [128 x 64] TMA box (the
 // K-major A operand, M = output dim) and the o_lat block's chunk as one bulk copy (the K-major B operand,
 // N = rows).  W^UV is an input of the decode call, never written by the kernels before this one in it, so
-// its first boxes are requested before the CTA waits for the merge.  The result is staged in shared memory
-// as bf16 rows and leaves as 16-byte stores (each output row is 256 contiguous bytes).
+// its first boxes are requested before the CTA waits for the merge.  With at most 64 rows (kRows = 64) the
+// eight stages hold the whole of W^UV_h, which is then all requested before the wait, and the o_lat chunks
+// all leave together after it.  The result is staged in shared memory as bf16 rows and leaves as 16-byte
+// stores (each output row is 256 contiguous bytes).
+template <int kRows, int kStages>
 __global__ void __launch_bounds__(kUpThreads) upproj_kernel(const __grid_constant__ CUtensorMap wuv_map,
                                                            const uint8_t* __restrict__ olat, int T, int H,
                                                            uint16_t* __restrict__ out, int32_t* dev_status) {
+    using Plan = UpPlan<kRows, kStages>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kUpOffBar);  // full[4], empty[4], done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kUpOffBar + 8 * (2 * kUpStages + 1));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Plan::kOffBar);  // full[kStages], empty[kStages], done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Plan::kOffBar + 8 * (2 * kStages + 1));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x;
-    const int t0 = blockIdx.y * kUpRows;
-    const int nt = min(kUpRows, T - t0);
+    const int t0 = blockIdx.y * kRows;
+    const int nt = min(kRows, T - t0);
     const int Tp = olat_rows(T);
-    const int NT = min(kUpRows, Tp - t0);  // rows of this o_lat block (a multiple of 16)
+    const int NT = min(kRows, Tp - t0);  // rows of this o_lat block (a multiple of 16)
     const uint32_t chunk_bytes = static_cast<uint32_t>(NT) * 128u;
     const uint8_t* blk = olat + (static_cast<int64_t>(h) * Tp + t0) * 1024;  // chunk c at c * NT * 128
     volatile int never = 0;
@@ -412,12 +431,12 @@ __global__ void __launch_bounds__(kUpThreads) upproj_kernel(const __grid_constan
         return;
     }
     if (tid == 0) {
-        for (int i = 0; i < 2 * kUpStages + 1; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 2 * kStages + 1; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         prefetch_tmap(&wuv_map);
-        for (int c = 0; c < kUpStages; ++c) {
+        for (int c = 0; c < kStages; ++c) {
             mbar_arrive_expect_tx(&bars[c], kWChunkBytes + chunk_bytes);
-            tma_load_3d(sbase + c * kUpStageBytes, &wuv_map, 0, h * 128, c, &bars[c]);
+            tma_load_3d(sbase + c * Plan::kStageBytes, &wuv_map, 0, h * 128, c, &bars[c]);
         }
     }
     if (warp == 0) tmem_alloc(tmem_slot, 256);
@@ -428,41 +447,42 @@ __global__ void __launch_bounds__(kUpThreads) upproj_kernel(const __grid_constan
     grid_dependency_wait();  // o_lat comes from the merge kernel
     bool ok = true;
     if (warp == 0 && lane == 0) {
-        // producer: the o_lat halves of the first four stages, then both halves of chunks 4..7 as stages free
+        // producer: the o_lat halves of the first kStages stages, then both halves of the remaining chunks (if
+        // any) as stages free
         const uint64_t once = l2_policy_evict_first();
-        for (int c = 0; c < kUpStages; ++c)
-            bulk_load_hint(sbase + c * kUpStageBytes + kUpOffB, blk + c * chunk_bytes, chunk_bytes, &bars[c], once);
-        for (int c = kUpStages; ok && c < 8; ++c) {
-            const int s = c % kUpStages;
-            ok = mbar_wait(&bars[kUpStages + s], 0, &never, kLimitNs);
+        for (int c = 0; c < kStages; ++c)
+            bulk_load_hint(sbase + c * Plan::kStageBytes + Plan::kOffB, blk + c * chunk_bytes, chunk_bytes, &bars[c], once);
+        for (int c = kStages; ok && c < 8; ++c) {
+            const int s = c % kStages;
+            ok = mbar_wait(&bars[kStages + s], 0, &never, kLimitNs);
             if (!ok) break;
             mbar_arrive_expect_tx(&bars[s], kWChunkBytes + chunk_bytes);
-            tma_load_3d(sbase + s * kUpStageBytes, &wuv_map, 0, h * 128, c, &bars[s]);
-            bulk_load_hint(sbase + s * kUpStageBytes + kUpOffB, blk + c * chunk_bytes, chunk_bytes, &bars[s], once);
+            tma_load_3d(sbase + s * Plan::kStageBytes, &wuv_map, 0, h * 128, c, &bars[s]);
+            bulk_load_hint(sbase + s * Plan::kStageBytes + Plan::kOffB, blk + c * chunk_bytes, chunk_bytes, &bars[s], once);
         }
         if (!ok) report(dev_status, MLA_DEVERR_TIMEOUT);
     } else if (warp == 1 && lane == 0) {
         // MMA issuer: out^T[d, t] += W^UV_h[d, chunk] o_lat[t, chunk], four K = 16 steps per chunk
         const uint32_t idesc = idesc_bf16_f32(128, NT, false, false);
         for (int c = 0; ok && c < 8; ++c) {
-            const int s = c % kUpStages;
-            ok = mbar_wait(&bars[s], static_cast<uint32_t>(c / kUpStages), &never, kLimitNs);
+            const int s = c % kStages;
+            ok = mbar_wait(&bars[s], static_cast<uint32_t>(c / kStages), &never, kLimitNs);
             if (!ok) break;
             tc_fence_after();
-            const uint64_t a0 = sdesc_sw128(sbase + s * kUpStageBytes, 16, 1024);
-            const uint64_t b0 = sdesc_sw128(sbase + s * kUpStageBytes + kUpOffB, 16, 1024);
+            const uint64_t a0 = sdesc_sw128(sbase + s * Plan::kStageBytes, 16, 1024);
+            const uint64_t b0 = sdesc_sw128(sbase + s * Plan::kStageBytes + Plan::kOffB, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_ss(tmem, a0 + static_cast<uint64_t>((kk * 32) >> 4), b0 + static_cast<uint64_t>((kk * 32) >> 4),
                        idesc, (c > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(smem_u32(&bars[kUpStages + s]));  // stage s free once these MMAs are done
+            mma_commit(smem_u32(&bars[kStages + s]));  // stage s free once these MMAs are done
         }
         if (!ok) report(dev_status, MLA_DEVERR_TIMEOUT);
-        mma_commit(smem_u32(&bars[2 * kUpStages]));  // also after a failure: TMEM is freed only once it fires
+        mma_commit(smem_u32(&bars[2 * kStages]));  // also after a failure: TMEM is freed only once it fires
     }
     ok = __syncthreads_and(ok);
     {
-        const bool done = mbar_wait(&bars[2 * kUpStages], 0, &never, kLimitNs);
+        const bool done = mbar_wait(&bars[2 * kStages], 0, &never, kLimitNs);
         __syncwarp();
         tc_fence_after();
         ok = __all_sync(0xffffffffu, done) && ok;
@@ -622,12 +642,21 @@ cudaError_t launch_upproj(const uint8_t* olat, const uint16_t* W_UV, int T, int 
                           cudaStream_t stream) {
     CUtensorMap map;
     if (!proj::weight_map(&map, W_UV, H)) return cudaErrorNotSupported;
-    cudaError_t e = cudaFuncSetAttribute(proj::upproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         proj::kUpSmemBytes);
+    if (T <= 64) {  // one block per head, the whole W^UV_h resident
+        using P = proj::UpPlan<64, 8>;
+        cudaError_t e = cudaFuncSetAttribute(proj::upproj_kernel<64, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             P::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        return proj::launch_pdl(proj::upproj_kernel<64, 8>, dim3(H, 1), proj::kUpThreads, P::kSmemBytes, stream, map,
+                                olat, T, H, out, dev_status);
+    }
+    using P = proj::UpPlan<proj::kOlatBlock, 4>;
+    cudaError_t e = cudaFuncSetAttribute(proj::upproj_kernel<proj::kOlatBlock, 4>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const dim3 grid(H, (T + proj::kUpRows - 1) / proj::kUpRows);
-    return proj::launch_pdl(proj::upproj_kernel, grid, proj::kUpThreads, proj::kUpSmemBytes, stream, map, olat, T, H,
-                            out, dev_status);
+    const dim3 grid(H, (T + proj::kOlatBlock - 1) / proj::kOlatBlock);
+    return proj::launch_pdl(proj::upproj_kernel<proj::kOlatBlock, 4>, grid, proj::kUpThreads, P::kSmemBytes, stream,
+                            map, olat, T, H, out, dev_status);
 }
 
 }  // namespace mla
