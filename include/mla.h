@@ -252,8 +252,11 @@ size_t mla_decode_workspace_bytes(int B, int n_q, int H, int num_splits);
  * The call launches the attend kernel (CTA pairs; for n_q * H <= 32 a kernel
  * that does a whole block on one SM), then the merge and up-projection
  * kernels (mla_decode_finish), each with programmatic stream serialization:
- * a kernel's set-up may overlap the end of the previous kernel on `stream`,
- * and it waits for that kernel to complete before reading any input.
+ * a kernel's set-up may overlap the end of the previous kernel on `stream`.
+ * The attend kernel waits for that kernel to complete before reading any
+ * input; the merge and up-projection kernels read kv_len and W_UV (inputs
+ * that no kernel of the call writes) before their wait, and everything the
+ * previous kernel of the call produced after it.
  * Errors: MLA_ERR_INVALID_ARG (null or misaligned pointer, bad scale, cap_blocks
  * or max_blocks < 1), MLA_ERR_UNSUPPORTED_SHAPE, MLA_ERR_WORKSPACE (ws_bytes
  * below mla_decode_workspace_bytes()), all before any launch; MLA_ERR_CUDA.
