@@ -14,17 +14,20 @@
 // absorb: one CTA per (128 latent columns, head, up to 128 query rows), so 4 CTAs share a
 // head and each moves a quarter of W^UK_h; the weight quarter lands as two TMA boxes
 // ([128 x 64] chunks, 128-byte swizzle) and is the MN-major A operand (M = latent
-// column, K = head dim) of 8 MMAs against the staged q_nope rows (N = rows).  (One CTA per
-// head with all four quarters measured slower: 15.1 against 13.6 us at T = 32, 68.9 against
-// 35.9 us at T = 256, ncu.)
-// merge: one CTA per (32 latent columns, sequence, row group), 1, 2 or 4 threads per row sharing
-// the sequence's pieces (the attend kernel writes them in [column group][row] order); it writes
-// o_lat into per-(head, 256-row block) tiles already in the swizzled K-major operand layout, so
-// each K step of the up-projection takes its operand with one bulk copy.
+// column, K = head dim) of 8 MMAs against the staged q_nope rows (N = rows).  The result
+// rows are staged in shared memory and leave as 16-byte stores.  (One CTA per head with all
+// four quarters measured slower: 15.1 against 13.6 us at T = 32, 68.9 against 35.9 us at
+// T = 256, ncu.)
+// merge: one CTA per (column slice, sequence, row group); the launch picks the threads per row
+// that share the sequence's pieces (1 to 16) and the slice width (8, 16 or 32 columns) from the
+// expected pieces per sequence and the grid size.  The attend kernel writes the pieces in
+// [column group][row] order; the merge writes o_lat into per-(head, 256-row block) tiles already
+// in the swizzled K-major operand layout, so each K step of the up-projection takes its operand
+// with one bulk copy.
 // upproj: one CTA per (head, up to 256 rows), the contraction over the latent columns streamed
-// through a four-stage ring; W^UV_h's first chunks are requested before the CTA waits for the
-// merge, so the weight load overlaps it.
-// upproj stages its bf16 result in shared memory and writes whole output rows with 16-byte stores.
+// through a ring of stages; W^UV_h's first chunks (all eight when T <= 64) are requested before
+// the CTA waits for the merge, so the weight load overlaps it.  The bf16 result is staged in
+// shared memory and whole output rows leave with 16-byte stores.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
